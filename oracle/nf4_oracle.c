@@ -1,0 +1,331 @@
+/*
+ * CPU oracle for the QLoRA NF4 + double-quantization linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the test suite, the package's smoke check and the
+ * bench's CPU-baseline / reference arm do.  It shares no code, header, table or
+ * constant with the CUDA path: the NF4 table is derived here from its quantile
+ * definition with this file's own inverse normal CDF.
+ *
+ * Every step is written to be read against the pages:
+ *   [p1] "QLoRAの理論と実装" (disassemble-channel.com)
+ *   [p2] Qiita article on why QLoRA survives 4-bit (TaiyoYamada)
+ * Quantisation follows the algorithm's steps in order (it is an encoding, so
+ * there is no shorter closed form); the linear layer is the plain definition
+ * evaluated in fp64 on the exact bf16 operands.
+ *
+ * Readings of points the pages leave open (all listed in the design notes):
+ *   - codebook: the p1 listing "create_nf4_codebook" (quantiles i/18, i=1..8 on
+ *     the negative side, j/16, j=9..15 on the positive side, zero pinned,
+ *     divided by the largest magnitude), because the p1 §5-1 formula with
+ *     i/(2^b+1), i=0 gives Phi^-1(0) = -inf;
+ *   - nearest code: exact argmin over the 16 levels, the lowest index winning
+ *     a tie (numpy argmin, p1 listing "quantize_nf4");
+ *   - w/absmax is one IEEE fp32 division;
+ *   - an all-zero block gets absmax 0 and code 8 (the level 0.0);
+ *   - nibble order: element 2j in the low nibble of byte j, row-major flatten;
+ *   - double quantization: linear unsigned 8-bit absmax quantization of each
+ *     group of 256 fp32 absmax constants, s2 = fp32(c2/255),
+ *     q = min(255, round-half-even(fp32(absmax/s2))), s2 == 0 gives q = 0;
+ *   - dequant: w = bf16( fp32( c[code] * fp32(q * s2) ) ).
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
+ * fp-contract is off so that no multiply-add is fused: every fp32 operation
+ * below rounds once, as written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_BLOCK 64   /* first-level block, p1 §5-1 step 1 and §5-2 */
+#define ORACLE_GROUP 256  /* second-level block of absmax constants, p1 §5-2 */
+
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Standard normal CDF and its inverse.                                      */
+/* Phi(x) = erfc(-x/sqrt(2)) / 2 and its upper tail 1 - Phi(x) =             */
+/* erfc(x/sqrt(2)) / 2 (textbook identities).  The inverse is found by       */
+/* bisection until the bracket is two adjacent doubles.  For p > 1/2 the     */
+/* upper tail is matched against 1 - p (exact for such p), so that no        */
+/* precision is lost to 1 - tiny.                                            */
+/* ------------------------------------------------------------------------ */
+static double oracle_phi(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
+static double oracle_phi_upper(double x) { return 0.5 * erfc(x / sqrt(2.0)); }
+
+double oracle_norm_ppf(double p) {
+    if (!(p > 0.0 && p < 1.0)) return NAN;
+    int upper = p > 0.5;
+    double target = upper ? 1.0 - p : p;
+    double lo = -40.0, hi = 40.0;
+    for (int it = 0; it < 4000; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if (mid <= lo || mid >= hi) break;  /* adjacent doubles */
+        /* both branches move lo up while mid is below the quantile */
+        int below = upper ? (oracle_phi_upper(mid) > target) : (oracle_phi(mid) < target);
+        if (below) lo = mid; else hi = mid;
+    }
+    double elo = upper ? fabs(oracle_phi_upper(lo) - target) : fabs(oracle_phi(lo) - target);
+    double ehi = upper ? fabs(oracle_phi_upper(hi) - target) : fabs(oracle_phi(hi) - target);
+    return (elo < ehi) ? lo : hi;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NF4 codebook.  [p1] "NF4量子化の仕組みの実装（教育目的）", listing         */
+/* create_nf4_codebook: eight negative levels at the quantiles i/18,        */
+/* i = 1..8, the level 0, seven positive levels at the quantiles j/16,      */
+/* j = 9..15; all divided by the largest magnitude; sorted ascending.       */
+/* This matches the "8 negative, 7 positive, zero pinned" statement of      */
+/* p1 §5-1 "数学的な構成".  out64 gets the fp64 levels, out32 their fp32     */
+/* rounding (the table the quantizer uses).                                  */
+/* ------------------------------------------------------------------------ */
+void oracle_nf4_codebook(double out64[16], float out32[16]) {
+    double v[16];
+    int n = 0;
+    for (int i = 1; i <= 8; ++i) v[n++] = oracle_norm_ppf((double)i / 18.0);
+    v[n++] = 0.0;
+    for (int j = 9; j <= 15; ++j) v[n++] = oracle_norm_ppf((double)j / 16.0);
+    double mx = 0.0;
+    for (int i = 0; i < 16; ++i) if (fabs(v[i]) > mx) mx = fabs(v[i]);
+    for (int i = 0; i < 16; ++i) v[i] = v[i] / mx;
+    /* insertion sort, ascending (the values are already ascending) */
+    for (int i = 1; i < 16; ++i) {
+        double t = v[i]; int j = i - 1;
+        while (j >= 0 && v[j] > t) { v[j + 1] = v[j]; --j; }
+        v[j + 1] = t;
+    }
+    for (int i = 0; i < 16; ++i) { out64[i] = v[i]; out32[i] = (float)v[i]; }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Nearest level.  [p1] §5-1 step 2: i* = argmin_i |w_norm - c_i|.  The     */
+/* distances are formed in fp64 from the fp32 operands; near any tie the     */
+/* two operands are within a factor 2^28 of each other (or one is 0), so the */
+/* differences are exact there and the comparison is the exact-real one.     */
+/* Strict '<' keeps the lowest index on a tie, as numpy's argmin does.      */
+/* ------------------------------------------------------------------------ */
+int oracle_nearest_code(float wn, const float table[16]) {
+    int best = 0;
+    double bd = fabs((double)wn - (double)table[0]);
+    for (int i = 1; i < 16; ++i) {
+        double d = fabs((double)wn - (double)table[i]);
+        if (d < bd) { bd = d; best = i; }
+    }
+    return best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Blockwise NF4 quantization, [p1] §5-1 steps 1-2 and the listing          */
+/* quantize_nf4 (semantics only): per block of 64 consecutive row-major     */
+/* elements, absmax = max |w| (exact); absmax == 0 leaves the block at 0;   */
+/* else w_norm = fp32(w / absmax) and the nearest level's index is stored   */
+/* in 4 bits.  n must be a multiple of 64 (every K is; the listing's zero    */
+/* padding of a ragged tail is therefore never exercised).                   */
+/* codes: n/2 bytes, absmax: n/64 floats.  Returns 0, or -1 on a bad n.     */
+/* ------------------------------------------------------------------------ */
+int oracle_quantize_nf4(const float* w, int64_t n, const float table[16],
+                        uint8_t* codes, float* absmax) {
+    if (n < 0 || n % ORACLE_BLOCK != 0) return -1;
+    int64_t nb = n / ORACLE_BLOCK;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) {
+        const float* blk = w + b * ORACLE_BLOCK;
+        float am = 0.0f;
+        for (int j = 0; j < ORACLE_BLOCK; ++j) {
+            float a = fabsf(blk[j]);
+            if (a > am) am = a;
+        }
+        absmax[b] = am;
+        uint8_t* out = codes + b * (ORACLE_BLOCK / 2);
+        for (int j = 0; j < ORACLE_BLOCK; j += 2) {
+            int c0, c1;
+            if (am == 0.0f) {
+                c0 = c1 = oracle_nearest_code(0.0f, table);
+            } else {
+                volatile float n0 = blk[j] / am;      /* one fp32 rounding */
+                volatile float n1 = blk[j + 1] / am;
+                c0 = oracle_nearest_code(n0, table);
+                c1 = oracle_nearest_code(n1, table);
+            }
+            out[j / 2] = (uint8_t)(c0 | (c1 << 4));   /* even element: low nibble */
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Double quantization.  [p1] §5-2 (the fp32 absmax constants of the first  */
+/* stage are quantized to 8 bits in blocks of 256) and [p2] "Double          */
+/* Quantization の仕組み" (W ~ (c2 * c1_quant) * W_quant).  Per group:       */
+/* c2 = max absmax, s2 = fp32(c2/255) is the stored fp32 second-level        */
+/* constant, q = min(255, rint_half_even(fp32(absmax/s2))), s2 == 0 -> q = 0.*/
+/* nb absmax values; the last group may be partial.                          */
+/* ------------------------------------------------------------------------ */
+void oracle_double_quant(const float* absmax, int64_t nb, uint8_t* q8, float* s2) {
+    int64_t ng = (nb + ORACLE_GROUP - 1) / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t g = 0; g < ng; ++g) {
+        int64_t b0 = g * ORACLE_GROUP;
+        int64_t b1 = b0 + ORACLE_GROUP < nb ? b0 + ORACLE_GROUP : nb;
+        float c2 = 0.0f;
+        for (int64_t b = b0; b < b1; ++b) if (absmax[b] > c2) c2 = absmax[b];
+        volatile float s = c2 / 255.0f;
+        s2[g] = s;
+        for (int64_t b = b0; b < b1; ++b) {
+            if (s == 0.0f) { q8[b] = 0; continue; }
+            volatile float ratio = absmax[b] / s;
+            float r = rintf(ratio);                 /* default mode: half-even */
+            if (r > 255.0f) r = 255.0f;
+            q8[b] = (uint8_t)r;
+        }
+    }
+}
+
+/* Round an fp32 value to bf16 (round to nearest, ties to even), returned as */
+/* its 16-bit pattern.  NaN stays a quiet NaN.                               */
+uint16_t oracle_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantization.  [p1] §5-1 step 3 (w_hat = c_i* x absmax), with the       */
+/* absmax rebuilt from the double-quantized pair as [p2] gives it            */
+/* (c1' = c2-scale x c1_quant), computed to bf16 as the storage/compute      */
+/* split of [p2] "4bitのまま計算しているわけではない" requires:               */
+/*   c1' = fp32(q * s2);  w32 = fp32(c[code] * c1');  w = bf16_rn(w32).      */
+/* out_f32 (may be NULL) gets w32, out_bf16 (may be NULL) gets w.           */
+/* ------------------------------------------------------------------------ */
+void oracle_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                    int64_t n, const float table[16], float* out_f32,
+                    uint16_t* out_bf16) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t b = i / ORACLE_BLOCK, g = b / ORACLE_GROUP;
+        int code = (i & 1) ? (codes[i / 2] >> 4) : (codes[i / 2] & 15);
+        volatile float c1 = (float)q8[b] * s2[g];
+        volatile float w32 = table[code] * c1;
+        if (out_f32) out_f32[i] = w32;
+        if (out_bf16) out_bf16[i] = oracle_f32_to_bf16(w32);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The linear layer in fp64, row-major.  W is N x K (out x in), X is M x K,  */
+/* A is r x K, B is N x r, s = alpha / r.                                    */
+/* [p1] "LoRAの復習" h = W0 x + (alpha/r) B A x, and "QLoRAの計算フロー"     */
+/* steps 1-4 (dequant, main product, A x then B, sum).  Column vectors of    */
+/* the pages become rows here: Y = X W^T + s (X A^T) B^T.                    */
+/* rows: if non-NULL, only those nrows rows of Y (and U) are computed and    */
+/* written compactly (row i of the output is row rows[i] of the full Y).     */
+/* ------------------------------------------------------------------------ */
+void oracle_linear_fwd(const double* X, const double* W, const double* A,
+                       const double* B, int64_t M, int64_t N, int64_t K, int r,
+                       double alpha, const int64_t* rows, int64_t nrows,
+                       double* Y, double* U) {
+    double s = alpha / (double)r;
+    int64_t count = rows ? nrows : M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const double* x = X + m * K;
+        double* u = U + i * r;
+        for (int j = 0; j < r; ++j) {               /* U = X A^T (r values) */
+            const double* a = A + (int64_t)j * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += x[k] * a[k];
+            u[j] = acc;
+        }
+        for (int64_t nn = 0; nn < N; ++nn) {        /* Y = X W^T + s U B^T */
+            const double* wr = W + nn * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += x[k] * wr[k];
+            double lora = 0.0;
+            for (int j = 0; j < r; ++j) lora += u[j] * B[nn * r + j];
+            Y[i * N + nn] = acc + s * lora;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward, [p1] "逆伝播と勾配の流れ":                                       */
+/*   dL/dB = (alpha/r) dL/dY (A X)^T   ->  dB = s dY^T U      (N x r)        */
+/*   dL/dA = (alpha/r) B^T dL/dY X^T   ->  dA = s (dY B)^T X  (r x K)        */
+/* W is frozen (no gradient).  dX is the chain rule through both paths:      */
+/*   dX = dY W + s (dY B) A                                   (M x K)        */
+/* Only dX's rows may be sampled (rows/nrows as in the forward); dA and dB   */
+/* are always full reductions over all M rows.                               */
+/* ------------------------------------------------------------------------ */
+void oracle_linear_bwd(const double* X, const double* W, const double* A,
+                       const double* B, const double* dY, int64_t M, int64_t N,
+                       int64_t K, int r, double alpha, const int64_t* rows,
+                       int64_t nrows, double* dX, double* dA, double* dB) {
+    double s = alpha / (double)r;
+    double* V = (double*)malloc(sizeof(double) * (size_t)M * (size_t)r);
+    double* U = (double*)malloc(sizeof(double) * (size_t)M * (size_t)r);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const double* dy = dY + m * N;
+        const double* x = X + m * K;
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;                        /* V = dY B */
+            for (int64_t nn = 0; nn < N; ++nn) acc += dy[nn] * B[nn * r + j];
+            V[m * r + j] = acc;
+            const double* a = A + (int64_t)j * K;   /* U = X A^T */
+            double au = 0.0;
+            for (int64_t k = 0; k < K; ++k) au += x[k] * a[k];
+            U[m * r + j] = au;
+        }
+    }
+    int64_t count = rows ? nrows : M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const double* dy = dY + m * N;
+        double* out = dX + i * K;
+        for (int64_t k = 0; k < K; ++k) out[k] = 0.0;
+        for (int64_t nn = 0; nn < N; ++nn) {         /* dY W */
+            double g = dy[nn];
+            const double* wr = W + nn * K;
+            for (int64_t k = 0; k < K; ++k) out[k] += g * wr[k];
+        }
+        for (int j = 0; j < r; ++j) {                /* + s V A */
+            double g = s * V[m * r + j];
+            const double* a = A + (int64_t)j * K;
+            for (int64_t k = 0; k < K; ++k) out[k] += g * a[k];
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k) {                /* dA = s V^T X */
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += V[m * r + j] * X[m * K + k];
+            dA[(int64_t)j * K + k] = s * acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t nn = 0; nn < N; ++nn) {             /* dB = s dY^T U */
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += dY[m * N + nn] * U[m * r + j];
+            dB[nn * r + j] = s * acc;
+        }
+    }
+    free(V);
+    free(U);
+}

@@ -1,0 +1,386 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+Sources of truth used here: values the pages print (tests/golden/closed_forms.json),
+two independent inverse-normal routines (Python's statistics.NormalDist and
+scipy.stats.norm), exact rational arithmetic (fractions.Fraction), numpy / torch
+library routines on special cases, finite differences, and algebraic identities.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+from statistics import NormalDist
+
+import numpy as np
+import pytest
+import torch
+from scipy.stats import norm
+
+import oracle
+from bit_nf4_quantized_quantize_b200 import synth
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")))
+
+
+# --------------------------------------------------------------------- table
+def test_inverse_normal_matches_two_libraries():
+    ps = np.concatenate([np.logspace(-12, -1, 23), np.linspace(0.05, 0.95, 37),
+                         1 - np.logspace(-12, -1, 23)])
+    nd = NormalDist()
+    for p in ps:
+        x = oracle.norm_ppf(p)
+        ref1 = nd.inv_cdf(float(p))
+        ref2 = float(norm.ppf(p))
+        assert abs(x - ref1) <= 1e-13 * max(1.0, abs(ref1)), (p, x, ref1)
+        assert abs(x - ref2) <= 1e-13 * max(1.0, abs(ref2)), (p, x, ref2)
+    assert abs(oracle.norm_ppf(0.5)) < 1e-15
+    for p in (0.1, 0.3, 1 / 18, 9 / 16):
+        assert abs(oracle.norm_ppf(p) + oracle.norm_ppf(1 - p)) < 1e-15
+
+
+def _page_listing_table_via_scipy():
+    """The codebook recipe of the page's create_nf4_codebook listing, run on scipy."""
+    neg = norm.ppf(np.linspace(1 / (2 * 9), 0.5, 8, endpoint=False))
+    pos = norm.ppf(np.linspace(0.5 + 1 / (2 * 8), 1 - 1 / (2 * 8), 7))
+    cb = np.concatenate([neg, [0.0], pos])
+    cb = cb / np.max(np.abs(cb))
+    return np.sort(cb)
+
+
+def _table_via_stdlib():
+    nd = NormalDist()
+    v = [nd.inv_cdf(i / 18) for i in range(1, 9)] + [0.0] + [nd.inv_cdf(j / 16) for j in range(9, 16)]
+    mx = max(abs(a) for a in v)
+    return np.sort(np.array(v) / mx)
+
+
+def test_codebook_matches_independent_constructions_bitwise_in_fp32():
+    t64, t32 = oracle.nf4_codebook()
+    for ref in (_page_listing_table_via_scipy(), _table_via_stdlib()):
+        assert np.max(np.abs(t64 - ref)) < 1e-15
+        assert np.array_equal(ref.astype(np.float32).view(np.uint32), t32.view(np.uint32))
+    # fp32 rounding is robust: every level sits far from an fp32 rounding boundary
+    for v in t64:
+        f = np.float32(v)
+        if v == 0:
+            continue
+        ulp = np.spacing(np.abs(f))
+        assert abs(float(f) - v) < 0.49 * float(ulp)
+
+
+def test_codebook_invariants_from_the_pages():
+    lv = GOLDEN["nf4_levels"]
+    t64, t32 = oracle.nf4_codebook()
+    assert t32.size == lv["total"]
+    assert np.all(np.diff(t64) > 0)
+    assert (t64 < 0).sum() == lv["negative"] and (t64 == 0).sum() == lv["zero"] \
+        and (t64 > 0).sum() == lv["positive"]
+    assert t32[0] == -1.0 and t32[8] == 0.0 and t32[15] < 1.0
+    # un-normalised levels are the quantiles i/18 and j/16
+    mx = abs(NormalDist().inv_cdf(1 / 18))
+    for i in range(8):
+        assert abs(t64[i] * mx - NormalDist().inv_cdf((i + 1) / 18)) < 1e-14
+    for j in range(7):
+        assert abs(t64[9 + j] * mx - NormalDist().inv_cdf((9 + j) / 16)) < 1e-14
+
+
+# ------------------------------------------------------------ nearest level
+def _exact_argmin(wn: float, table32):
+    q = Fraction(float(wn))
+    d = [abs(q - Fraction(float(c))) for c in table32]
+    m = min(d)
+    return d.index(m)
+
+
+def test_nearest_code_is_exact_argmin_lowest_index_on_ties():
+    _, t32 = oracle.nf4_codebook()
+    probes = [np.float32(v) for v in np.linspace(-1, 1, 801)]
+    g = np.random.default_rng(7)
+    probes += [np.float32(v) for v in g.uniform(-1, 1, 400)]
+    # fp32 neighbours of every exact midpoint, where a naive fp32 search can differ
+    for i in range(15):
+        mid = (float(t32[i]) + float(t32[i + 1])) / 2
+        f = np.float32(mid)
+        for k in range(-3, 4):
+            v = f
+            step = np.float32(np.inf) if k > 0 else np.float32(-np.inf)
+            for _ in range(abs(k)):
+                v = np.nextafter(v, step)
+            probes.append(np.float32(v))
+    probes += [np.float32(0.0), np.float32(-0.0), np.float32(1e-40), np.float32(-1e-40),
+               np.float32(1.0), np.float32(-1.0)]
+    for p in probes:
+        assert oracle.nearest_code(float(p), t32) == _exact_argmin(float(p), t32), p
+
+
+def test_nearest_code_tie_goes_to_lower_index():
+    # a table where an fp32 value lies exactly on a midpoint: levels 0.25 and 0.5
+    t = np.array([-1.0, -0.5, -0.25, 0.0, 0.25, 0.5, 0.75, 1.0] + [2.0 + i for i in range(8)],
+                 np.float32)
+    assert oracle.nearest_code(0.375, t) == 4
+    assert oracle.nearest_code(float(np.nextafter(np.float32(0.375), np.float32(1))), t) == 5
+    assert oracle.nearest_code(-0.375, t) == 1
+
+
+# ----------------------------------------------------------------- quantize
+def test_round_trip_of_every_table_value():
+    _, t32 = oracle.nf4_codebook()
+    blk = np.repeat(t32, 4).astype(np.float32)          # absmax 1 (from c_0 = -1)
+    codes, absmax = oracle.quantize_nf4(blk)
+    assert absmax[0] == 1.0
+    unpacked = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    assert np.array_equal(unpacked, np.repeat(np.arange(16), 4))
+    # with DQ: c2 = 1 -> s2 = fp32(1/255) and fp32(255 * s2) == 1 exactly
+    q8, s2 = oracle.double_quant(absmax)
+    assert q8[0] == 255 and s2[0] == np.float32(1) / np.float32(255)
+    assert np.float32(255) * s2[0] == np.float32(1)
+    w32, wb = oracle.dequant(codes, q8, s2, 64)
+    assert np.array_equal(w32.view(np.uint32), blk.view(np.uint32))
+    # bf16 conversion matches torch's round-to-nearest-even
+    tb = torch.from_numpy(blk.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(wb, tb)
+
+
+def test_nibble_order_and_zero_block_and_layout():
+    blk = np.zeros(128, np.float32)
+    blk[0], blk[1] = -1.0, 1.0
+    codes, absmax = oracle.quantize_nf4(blk)
+    assert codes[0] == (0 | (15 << 4)) and codes[1] == 0x88
+    assert absmax[0] == 1.0 and absmax[1] == 0.0
+    assert np.all(codes[32:] == 0x88)                    # all-zero block -> level 0.0 (code 8)
+
+
+def test_requantize_dequantized_codes_is_identity():
+    _, t32 = oracle.nf4_codebook()
+    g = np.random.default_rng(3)
+    nblk = 512
+    codes = g.integers(0, 16, size=(nblk, 64))
+    codes[:, g.integers(0, 64, nblk)] = 0                # every block holds code 0 -> absmax
+    codes[np.arange(nblk), g.integers(0, 64, nblk)] = 0
+    scale = g.uniform(1e-3, 10.0, nblk).astype(np.float32)
+    w = (t32[codes] * scale[:, None]).astype(np.float32).reshape(-1)
+    c2, am = oracle.quantize_nf4(w)
+    un = np.stack([c2 & 15, c2 >> 4], 1).reshape(nblk, 64)
+    assert np.array_equal(un, codes)
+    assert np.array_equal(am, scale)
+
+
+def test_power_of_two_scaling_is_exact():
+    x = synth.normal_f32(synth.rng(9, 0), (64 * 40,), 0.02)
+    c1, a1 = oracle.quantize_nf4(x)
+    for e in (-20, -3, 5, 30):
+        c2, a2 = oracle.quantize_nf4((x * np.float32(2.0 ** e)).astype(np.float32))
+        assert np.array_equal(c1, c2)
+        assert np.array_equal(a2, (a1 * np.float32(2.0 ** e)).astype(np.float32))
+
+
+def test_quantize_brute_force_tiny():
+    """Brute force over all 16 levels with exact rationals on the tiny workload's first rows."""
+    _, t32 = oracle.nf4_codebook()
+    w = synth.weight(1, 0, 256, 256)[:4].reshape(-1)     # 1024 values, 16 blocks
+    codes, absmax = oracle.quantize_nf4(w)
+    un = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    for b in range(w.size // 64):
+        blk = w[b * 64:(b + 1) * 64]
+        am = max(abs(float(v)) for v in blk)
+        assert absmax[b] == np.float32(am)
+        for j, v in enumerate(blk):
+            n = np.float32(v) / np.float32(am)           # IEEE fp32 division (numpy)
+            assert un[b * 64 + j] == _exact_argmin(float(n), t32)
+
+
+def test_nf4_beats_int4_on_normal_data():
+    """Sanity from the pages: NF4's MSE is roughly 10-30% below uniform INT4 (N(0,1), block 64)."""
+    spec = GOLDEN["nf4_vs_int4_mse_improvement_percent"]
+    g = synth.rng(42, 0)
+    w = g.standard_normal(spec["samples"] - spec["samples"] % 64).astype(np.float32)
+    codes, absmax = oracle.quantize_nf4(w)
+    _, t32 = oracle.nf4_codebook()
+    un = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    w_nf4 = t32[un].astype(np.float64) * np.repeat(absmax.astype(np.float64), 64)
+    lv = np.linspace(-1, 1, 16)
+    wb = w.reshape(-1, 64).astype(np.float64)
+    am = np.abs(wb).max(1, keepdims=True)
+    idx = np.abs(wb[:, :, None] / am[:, :, None] - lv[None, None, :]).argmin(-1)
+    w_int4 = (lv[idx] * am).reshape(-1)
+    mse_nf4 = np.mean((w - w_nf4) ** 2)
+    mse_int4 = np.mean((w - w_int4) ** 2)
+    imp = 100 * (1 - mse_nf4 / mse_int4)
+    assert spec["low"] - 5 <= imp <= spec["high"] + 5, imp
+
+
+# ---------------------------------------------------------- double quant
+def test_double_quant_hand_cases():
+    c2 = np.float32(0.037)
+    a = np.array([c2] * 256, np.float32)
+    q8, s2 = oracle.double_quant(a)
+    assert np.all(q8 == 255) and s2[0] == c2 / np.float32(255)
+    a = np.zeros(256, np.float32)
+    a[0], a[1] = c2, c2 / np.float32(2)
+    q8, s2 = oracle.double_quant(a)
+    s = Fraction(float(s2[0]))
+    half = Fraction(float(np.float32(np.float32(c2 / np.float32(2)) / s2[0])))
+    exp = int(half.__round__())                           # Fraction rounds half to even
+    assert q8[0] == 255 and q8[1] == exp and np.all(q8[2:] == 0)
+    assert s == Fraction(float(np.float32(c2) / np.float32(255)))
+
+
+def test_double_quant_error_bound_and_partial_group():
+    g = np.random.default_rng(11)
+    a = np.abs(g.normal(0, 0.05, 256 * 7 + 100)).astype(np.float32)   # ragged last group
+    q8, s2 = oracle.double_quant(a)
+    assert s2.size == 8
+    for i, v in enumerate(a):
+        s = float(s2[i // 256])
+        rec = float(np.float32(np.float32(q8[i]) * s2[i // 256]))
+        assert abs(rec - float(v)) <= s / 2 * (1 + 1e-6) + 1e-12
+        grp = a[(i // 256) * 256:(i // 256 + 1) * 256]
+        assert s2[i // 256] == np.float32(grp.max()) / np.float32(255)
+
+
+def test_double_quant_zero_and_subnormal_groups():
+    q8, s2 = oracle.double_quant(np.zeros(256, np.float32))
+    assert s2[0] == 0 and np.all(q8 == 0)
+    tiny = np.full(256, np.float32(1e-44), np.float32)    # c2/255 underflows to 0
+    q8, s2 = oracle.double_quant(tiny)
+    assert s2[0] == 0 and np.all(q8 == 0)
+
+
+# ---------------------------------------------------------------- overhead
+def test_overheads_match_the_pages_closed_forms():
+    G = GOLDEN
+    sq = 32 / 64
+    dq = 4 + 8 / 64 + 32 / (64 * 256)
+    assert sq == G["single_quant_overhead_bit_per_param"]["value"]
+    assert 4 + sq == G["single_quant_total_bit_per_param"]["value"]
+    assert 8 / 64 == G["double_quant_second_term_bit_per_param"]["value"]
+    assert abs(32 / (64 * 256) - G["double_quant_third_term_bit_per_param_approx"]["value"]) \
+        <= G["double_quant_third_term_bit_per_param_approx"]["tolerance_abs"]
+    assert abs(dq - G["double_quant_total_bit_per_param_approx"]["value"]) <= 5e-4
+    saving = 4.5 - dq
+    assert saving == 0.373046875
+    assert abs(saving - G["dq_saving_bit_per_param_approx"]["value"]) <= 5e-3
+    assert abs(65e9 * sq / 8 / 1e9 - 4.0) <= 0.1
+    assert abs(65e9 * saving / 8 / 1e9 - 3.0) <= 0.1
+    # the buffers the oracle produces have exactly that size, for every workload shape
+    for shape in [(256, 256), (4096, 4096), (11008, 4096), (4096, 11008), (8192, 8192),
+                  (22016, 8192)]:
+        n = shape[0] * shape[1]
+        nb = n // 64
+        bytes_ = n // 2 + nb + 4 * ((nb + 255) // 256)
+        assert 8 * bytes_ / n == dq
+    w = synth.weight(1, 0, 256, 256)
+    codes, q8, s2, _ = oracle.quantize_nf4_dq(w.reshape(-1))
+    assert 8 * (codes.nbytes + q8.nbytes + s2.nbytes) / w.size == dq
+
+
+def test_lora_parameter_counts():
+    G = GOLDEN
+    d = k = 4096
+    assert 8 * (d + k) == G["lora_params_d4096_k4096_r8"]["value"]
+    assert d * k == G["dense_params_d4096_k4096"]["value"]
+    assert abs(100 * 8 * (d + k) / (d * k) - 0.4) <= 0.05
+    assert 4 * 2 * 4096 * 64 * 32 == G["lora_params_7b_attention_r64"]["value"]
+
+
+# --------------------------------------------------------------- bf16 / dequant
+def test_bf16_rounding_matches_torch():
+    g = np.random.default_rng(5)
+    x = np.concatenate([g.normal(0, 1, 5000), g.normal(0, 1e-30, 200), [0.0, -0.0, 1e38, -3e-39]])
+    x = x.astype(np.float32)
+    # values exactly halfway between two bf16 numbers (tie -> even)
+    ties = (np.arange(1, 200, dtype=np.uint32) << np.uint32(16)) | np.uint32(0x8000)
+    x = np.concatenate([x, ties.view(np.float32) + 0])
+    ours = oracle.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_dequant_matches_formula_in_fp32_numpy():
+    w = synth.weight(1, 0, 256, 256).reshape(-1)
+    codes, q8, s2, _ = oracle.quantize_nf4_dq(w)
+    _, t32 = oracle.nf4_codebook()
+    w32, wb = oracle.dequant(codes, q8, s2, w.size)
+    un = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    c1 = (q8.astype(np.float32) * np.repeat(s2, 256)[: q8.size]).astype(np.float32)
+    ref = (t32[un] * np.repeat(c1, 64)).astype(np.float32)
+    assert np.array_equal(w32.view(np.uint32), ref.view(np.uint32))
+    tb = torch.from_numpy(ref.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(wb, tb)
+    # reconstruction error: within half a level spacing times absmax plus the DQ error
+    assert np.max(np.abs(w32 - w)) < 0.2 * np.abs(w).max()
+
+
+# ----------------------------------------------------------------- linear
+def _small_case(M=9, N=24, K=64, r=3, seed=0):
+    g = np.random.default_rng(seed)
+    return (g.normal(size=(M, K)), g.normal(size=(N, K)) * 0.1, g.normal(size=(r, K)) / 8,
+            g.normal(size=(N, r)) * 0.1, g.normal(size=(M, N)))
+
+
+def test_fwd_special_cases_and_merge_identity():
+    X, W, A, B, _ = _small_case()
+    alpha = 5.0
+    s = alpha / A.shape[0]
+    Y, U = oracle.linear_fwd(X, W, A, np.zeros_like(B), alpha)
+    assert np.allclose(Y, X @ W.T, rtol=1e-13, atol=1e-13)
+    Y, U = oracle.linear_fwd(X, W, A, B, alpha)
+    # merging the adapter into the dense weight gives the same layer
+    assert np.allclose(Y, X @ (W + s * B @ A).T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(U, X @ A.T, rtol=1e-13, atol=1e-13)
+    rows = np.array([7, 0, 3])
+    Yr, Ur = oracle.linear_fwd(X, W, A, B, alpha, rows=rows)
+    assert np.array_equal(Yr, Y[rows]) and np.array_equal(Ur, U[rows])
+
+
+def test_bwd_against_finite_differences_and_adjoint():
+    X, W, A, B, dY = _small_case(M=5, N=8, K=6, r=2, seed=1)
+    alpha = 3.0
+
+    def loss(A_, B_, X_=X):
+        return float(np.sum(dY * oracle.linear_fwd(X_, W, A_, B_, alpha)[0]))
+
+    dX, dA, dB = oracle.linear_bwd(X, W, A, B, dY, alpha)
+    h = 1e-6
+    for idx in np.ndindex(A.shape):
+        Ap, Am = A.copy(), A.copy()
+        Ap[idx] += h
+        Am[idx] -= h
+        assert abs((loss(Ap, B) - loss(Am, B)) / (2 * h) - dA[idx]) < 1e-7
+    for idx in np.ndindex(B.shape):
+        Bp, Bm = B.copy(), B.copy()
+        Bp[idx] += h
+        Bm[idx] -= h
+        assert abs((loss(A, Bp) - loss(A, Bm)) / (2 * h) - dB[idx]) < 1e-7
+    for idx in [(0, 0), (2, 3), (4, 5)]:
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        assert abs((loss(A, B, Xp) - loss(A, B, Xm)) / (2 * h) - dX[idx]) < 1e-7
+    # the layer is linear in X: <dY, Y(X)> == <dX, X>
+    Y, _ = oracle.linear_fwd(X, W, A, B, alpha)
+    assert abs(np.sum(dY * Y) - np.sum(dX * X)) < 1e-10 * max(1, abs(np.sum(dY * Y)))
+
+
+def test_bwd_zero_adapter_and_rows():
+    X, W, A, B, dY = _small_case(M=7, N=16, K=64, r=4, seed=2)
+    dX, dA, dB = oracle.linear_bwd(X, W, A, np.zeros_like(B), dY, 8.0)
+    assert np.allclose(dX, dY @ W, rtol=1e-13, atol=1e-13)
+    assert np.all(dA == 0)
+    assert np.allclose(dB, 2.0 * dY.T @ (X @ A.T), rtol=1e-12, atol=1e-12)
+    dX, dA, dB = oracle.linear_bwd(X, W, A, B, dY, 8.0)
+    dXr, dAr, dBr = oracle.linear_bwd(X, W, A, B, dY, 8.0, rows=np.array([6, 1]))
+    assert np.array_equal(dXr, dX[[6, 1]]) and np.array_equal(dAr, dA) and np.array_equal(dBr, dB)
+
+
+def test_oracle_rejects_ragged_length():
+    with pytest.raises(ValueError):
+        oracle.quantize_nf4(np.zeros(65, np.float32))
+
+
+def test_planted_mistake_is_caught():
+    """A plausible slip (dropping the alpha/r scale on the adapter) fails the merge identity."""
+    X, W, A, B, _ = _small_case()
+    Y, _ = oracle.linear_fwd(X, W, A, B, 5.0)
+    wrong = X @ (W + B @ A).T
+    assert not np.allclose(Y, wrong, rtol=1e-6, atol=1e-6)
