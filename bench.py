@@ -1,0 +1,410 @@
+#!/usr/bin/env python3
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+Workload (one GPU): a single 4096 x 4096 frozen layer, NF4 + double quant,
+M = 4096 tokens (4 x 1024), LoRA r = 64, alpha = 16, seeded synthetic inputs
+(W ~ N(0, 0.02^2), X, dY ~ N(0, 1), A ~ N(0, 1/4096), B ~ N(0, 0.01^2)).
+One step = the whole hot path once: quantize + double-quantize W, forward
+(U = X A^T, Y = X dequant(W)^T + s U B^T), backward (V, dX, dA, dB).
+
+Metric: algorithmic fwd+bwd FLOP of the step / device time of the step
+(TFLOP/s); the quantize GB/s and per-kernel times are reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun as independent replicas (one process per GPU, no
+collective on the data path; weak scaling).  --impl reference times the CPU
+oracle on the same workload (a bounded sample of it per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "train4096"
+N_OUT, K_IN, M_TOK, RANK, ALPHA = 4096, 4096, 4096, 64, 16.0
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and quantize GB/s; % of roofline vs CPU oracle"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+CPU_SAMPLE_TOKENS = 512       # cpu_baseline: tokens of the oracle's sample step
+REF_SAMPLE_TOKENS = 128       # --impl reference: tokens per sampled step
+
+
+def step_flops(M, N, K, r):
+    """Algorithmic FLOP of fwd + bwd: main 4MNK, LoRA fwd 2Mr(K+N), LoRA bwd 2Mr(N+K) + 2rMK + 2NMr."""
+    return 4 * M * N * K + 2 * M * r * (K + N) + 2 * M * r * (N + K) + 2 * r * M * K + 2 * N * M * r
+
+
+def quant_bytes(N, K):
+    """Algorithmic quantize traffic: fp32 W in, packed codes + q8 + s2 out."""
+    n = N * K
+    nb = n // 64
+    return 4 * n + n // 2 + nb + 4 * ((nb + 255) // 256)
+
+
+def kernel_flops(kind, M, N, K, r):
+    if kind == "fwd_fused":
+        return 2 * M * N * K + 2 * M * N * r
+    if kind == "dx_fused":
+        return 2 * M * N * K + 2 * M * K * r
+    return None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_quantize_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kind):
+    """Per-launch DRAM bytes of `kind` from the committed ncu summary, if it matches these sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kind)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def make_inputs(M=M_TOK, N=N_OUT, K=K_IN, r=RANK, alpha=ALPHA):
+    from bit_nf4_quantized_quantize_b200 import synth
+    return synth.layer_inputs(WORKLOAD, M=M, shape=(N, K), r=r, alpha=alpha)
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_step(inp, M_s):
+    """One sampled step on the CPU oracle: quantize the whole W, then fwd + bwd on M_s tokens."""
+    import oracle
+    from bit_nf4_quantized_quantize_b200 import synth
+    N, K, r, alpha = inp["N"], inp["K"], inp["r"], inp["alpha"]
+    t0 = time.perf_counter()
+    codes, q8, s2, _ = oracle.quantize_nf4_dq(inp["W"].reshape(-1))
+    t1 = time.perf_counter()
+    _, wb = oracle.dequant(codes, q8, s2, N * K)
+    What = synth.bf16_bits_to_f32(wb).astype(np.float64).reshape(N, K)
+    f = lambda k: synth.bf16_bits_to_f32(inp[k]).astype(np.float64)
+    X, A, B, dY = f("X")[:M_s], f("A"), f("B"), f("dY")[:M_s]
+    t2 = time.perf_counter()
+    oracle.linear_fwd(X, What, A, B, alpha)
+    oracle.linear_bwd(X, What, A, B, dY, alpha)
+    t3 = time.perf_counter()
+    return dict(quant_s=t1 - t0, linear_s=t3 - t2, total_s=(t1 - t0) + (t3 - t2))
+
+
+def cpu_baseline(inp):
+    import oracle
+    N, K, r = inp["N"], inp["K"], inp["r"]
+    t = oracle_step(inp, CPU_SAMPLE_TOKENS)
+    fl = step_flops(CPU_SAMPLE_TOKENS, N, K, r)
+    return {"value": fl / t["linear_s"] / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": (f"oracle fwd+bwd on {CPU_SAMPLE_TOKENS} of the {M_TOK} tokens (fp64, full N=K=4096, r=64) "
+                       f"took {t['linear_s']:.2f} s; quantize+DQ of the full 4096x4096 W took {t['quant_s']:.2f} s "
+                       f"= {quant_bytes(N, K) / t['quant_s'] / 1e9:.3f} GB/s"),
+            "quantize_gbs": quant_bytes(N, K) / t["quant_s"] / 1e9}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    inp = make_inputs()
+    N, K, r = inp["N"], inp["K"], inp["r"]
+    for _ in range(args.warmup):
+        oracle_step(inp, REF_SAMPLE_TOKENS)
+    times = [oracle_step(inp, REF_SAMPLE_TOKENS) for _ in range(args.steps)]
+    lin = sum(t["linear_s"] for t in times) / len(times)
+    qs = sum(t["quant_s"] for t in times) / len(times)
+    fl = step_flops(REF_SAMPLE_TOKENS, N, K, r)
+    value = fl / lin / 1e12
+    sample = (f"each step: oracle quantize+DQ of the full 4096x4096 W ({qs:.2f} s) and fp64 fwd+bwd on "
+              f"{REF_SAMPLE_TOKENS} of the {M_TOK} tokens ({lin:.2f} s); value = that sample's FLOP / its time")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": (lin + qs) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "train4096: one 4096x4096 NF4+DQ layer, M=4096 tokens, r=64, alpha=16; "
+                                   "step = quantize + fwd + bwd (sampled tokens on the CPU)",
+                       "N": N_OUT, "K": K_IN, "M": M_TOK, "r": RANK, "alpha": ALPHA},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "quantize_gbs": quant_bytes(N, K) / qs / 1e9}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------- GPU
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import bit_nf4_quantized_quantize_b200 as q
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    q.load()
+    inp = make_inputs()
+    N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
+
+    def pinned(a, dtype=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dtype is not None:
+            t = t.view(dtype)
+        return t.pin_memory()
+
+    hW = pinned(inp["W"])
+    hX, hA, hB, hdY = (pinned(inp[k].view(np.int16), torch.bfloat16) for k in ("X", "A", "B", "dY"))
+    W, X, A, B, dY = (t.to(dev) for t in (hW, hX, hA, hB, hdY))
+    nc, nb, ng = q._binding.quant_sizes(N, K)
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+    q8 = torch.empty(nb, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(ng, dtype=torch.float32, device=dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(Wd=W, Xd=X, dYd=dY, Ad=A, Bd=B):
+        q.qlora_quantize_nf4_dq(Wd, codes, q8, s2)
+        q.qlora_linear_fwd(codes, q8, s2, N, K, Xd, Ad, Bd, alpha, Y=Y, U_save=U, workspace=ws)
+        q.qlora_linear_bwd(codes, q8, s2, N, K, Xd, Ad, Bd, alpha, dYd, U_saved=U, dX=dX, dA=dA, dB=dB,
+                           workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        step()
+    torch.cuda.synchronize()
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {q.qlora_strerror(rc)}")
+
+    # ---------------------------------------------------------------- timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    q.qlora_timing_enable(True)
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(float(i))          # L2 flush between steps, outside the step's events
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    barrier()
+    kern = q.qlora_timing_collect()
+    q.qlora_timing_enable(False)
+    clocks = sampler.stop()
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the timed region: {q.qlora_strerror(rc)}")
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    launches = sum(c for _, c in kern.values())
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    n_e2e = max(3, min(args.steps, 10))
+    hY = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    hdX = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
+    hdA = torch.empty(r, K, dtype=torch.float32).pin_memory()
+    hdB = torch.empty(N, r, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
+    d2h = sum(t.numel() * t.element_size() for t in (hY, hdX, hdA, hdB))
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(n_e2e):
+        flush.fill_(float(i))
+        e_ev[i][0].record()
+        W.copy_(hW, non_blocking=True)
+        X.copy_(hX, non_blocking=True)
+        A.copy_(hA, non_blocking=True)
+        B.copy_(hB, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        step()
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(dX, non_blocking=True)
+        hdA.copy_(dA, non_blocking=True)
+        hdB.copy_(dB, non_blocking=True)
+        e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e_ev) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        return
+    fl = step_flops(M, N, K, r)
+    value = world * fl / (step_ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    per_step = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps,
+                    "ms_per_launch": v[0] / v[1]} for k, v in kern.items()}
+    dom = max(kern, key=lambda k: kern[k][0])
+    dom_ms = kern[dom][0] / kern[dom][1]
+    kf = kernel_flops(dom, M, N, K, r)
+    long_region = wall > 1.0
+    if kf is not None:
+        peak = peaks["bf16_sustained"] if long_region else peaks["bf16"]
+        achieved = kf / (dom_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": load_traffic(dom),
+                "peak_source": f"{peaks['source']} bf16 dense "
+                               f"{'sustained' if long_region else 'burst'} (timed region {wall:.2f} s)",
+                "algorithmic_flop_per_launch": kf, "ms_per_launch": dom_ms}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": load_traffic(dom)}
+    qk = kern.get("quantize")
+    quant_gbs = quant_bytes(N, K) / (qk[0] / qk[1] * 1e-3) / 1e9 if qk else None
+    fwd_ms = sum(per_step[k]["ms_per_step"] for k in per_step if k in ("lora_gemm", "lora_reduce", "fwd_fused")) / 1
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "train4096: one 4096x4096 NF4+DQ layer, M=4096 tokens (4x1024), r=64, alpha=16; "
+                               "step = quantize + fwd + bwd",
+                   "N": N, "K": K, "M": M, "r": r, "alpha": alpha,
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the step events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": roof,
+        "quantize": {"gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
+                     "frac": quant_gbs / peaks["hbm_gbs"] if quant_gbs else None,
+                     "algorithmic_bytes": quant_bytes(N, K), "traffic": load_traffic("quantize")},
+        "kernels": per_step,
+        "gpu_launches": launches,
+        "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

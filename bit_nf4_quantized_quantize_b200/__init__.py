@@ -1,0 +1,28 @@
+"""QLoRA NF4 + double-quant linear layer for one B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libqlora_nf4.so`` (declared in
+``include/qlora_nf4.h``).  Every function here only marshals arguments: torch
+tensors supply device memory and the current CUDA stream, and every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback: if
+the library is missing or no sm_100 device is current, calls raise.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    QLORA_OUT_BF16,
+    QLORA_OUT_FP32,
+    QloraError,
+    exported_symbols,
+    lib_path,
+    load,
+    qlora_dequant,
+    qlora_device_status,
+    qlora_linear_bwd,
+    qlora_linear_fwd,
+    qlora_nf4_codebook,
+    qlora_quantize_nf4_dq,
+    qlora_strerror,
+    qlora_timing_collect,
+    qlora_timing_enable,
+    qlora_workspace_bytes,
+)

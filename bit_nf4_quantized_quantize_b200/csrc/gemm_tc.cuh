@@ -1,0 +1,452 @@
+// tcgen05 (5th-generation tensor core) GEMM for the QLoRA linear layer, sm_100a.
+//
+// D[128 x BN] tile (+)= A[128 x K] * B[BN x K]^T with bf16 operands staged in
+// 128-byte-swizzled shared memory and an fp32 accumulator in TMEM.  One
+// template covers every product of the layer:
+//
+//   forward   Y  = X dequant(W)^T + (s U) B^T      B operand = NF4 weight, K-major
+//   backward  dX = dY dequant(W)  + (s V) A        B operand = NF4 weight, MN-major
+//   LoRA      U  = X A^T, V = dY B                 split-K, fp32 partials
+//   grads     dA^T = X^T V, dB = dY^T U            split-M, fp32 partials
+//
+// For the two weight products the B tile is never read from HBM in bf16: the
+// producer warp streams the packed 4-bit codes with TMA, the dequant warps
+// expand them in registers (one 16-entry bf16 table per 64-block, looked up
+// with byte permutes) and write the bf16 tile straight into the swizzled
+// layout UMMA reads.  The adapter term runs as extra K=64 slices of the same
+// accumulator (U or V pre-scaled by s on the A side, B or A on the B side), so
+// the LoRA up-projection costs no separate pass over Y.
+//
+// Warp roles (64 + 32*NDW threads):
+//   warp 0        TMA producer (one elected lane)
+//   warp 1        TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..     dequant (weight products), then epilogue (TMEM -> registers
+//                 -> global).  Warp w reads TMEM lanes 32*(w%4)...
+// Pipelines: full_tma[s] (TMA bytes landed), full_w[s] (dequant wrote the B
+// tile), empty[s] (the MMAs that read stage s completed), accum_full.  Every
+// wait is bounded (ptx_sm100.cuh): on expiry the CTA latches the device error
+// flag, every role leaves its loop, TMEM is freed and the CTA exits.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "ptx_sm100.cuh"
+
+namespace qlora {
+
+enum BSource : int {
+  kBTmaK = 0,    // B tile loaded by TMA, K-major
+  kBTmaMN = 1,   // B tile loaded by TMA, MN-major
+  kBDeqK = 2,    // B = dequant(W) rows (weight row n = B row), K-major   (forward)
+  kBDeqMN = 3,   // B = dequant(W)^T (weight row = reduction index), MN-major (dX)
+};
+enum OutMode : int { kOutBf16 = 0, kOutF32Partial = 1 };
+
+constexpr int kBK = 64;                 // reduction elements per stage (128 B of bf16)
+constexpr int kBM = 128;                // MMA M
+constexpr int kATileBytes = kBM * kBK * 2;
+
+struct GemmArgs {
+  int m_rows;             // rows of D (MMA M side) in total
+  int n_cols;             // columns of D in total
+  int k_steps;            // main reduction steps (of 64) in total
+  int steps_per_split;    // main steps per CTA along blockIdx.z
+  int n_lora;             // adapter slices (of 64) issued before the main steps
+  // NF4 weight (dequant sources only)
+  const uint8_t* q8;
+  const float* s2;
+  int w_rows;             // N of the weight
+  int w_kblocks;          // K/64 of the weight
+  float level[16];        // NF4 levels (fp32)
+  // output
+  void* out;
+  int64_t ld_out;         // elements between consecutive D rows
+  int64_t split_stride;   // elements between splits (partial mode)
+};
+
+template <int BN, int NSTAGE, int BSRC, int NDW>
+struct GemmSmem {
+  static constexpr bool kDeq = (BSRC == kBDeqK || BSRC == kBDeqMN);
+  static constexpr int kBTileBytes = BN * kBK * 2;
+  static constexpr int kPTileBytes = kDeq ? BN * kBK / 2 : 0;
+  static constexpr int kAOff = 0;
+  static constexpr int kBOff = kAOff + NSTAGE * kATileBytes;
+  static constexpr int kPOff = kBOff + NSTAGE * kBTileBytes;
+  static constexpr int kBarOff = kPOff + NSTAGE * kPTileBytes;
+  static constexpr int kNumBars = 3 * NSTAGE + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kDynBytes = kBytes + 1024;  // slack to align the base to 1024 B
+};
+
+// ---------------------------------------------------------------------------
+// Register-level NF4 expansion.  For one 64-block with combined scale c1, the
+// 16 values bf16(fp32(level[i] * c1)) are split into low bytes (lo[0..3]) and
+// high bytes (hi[0..3]), 4 per register; a byte permute then looks up 4 codes
+// at once.
+struct DeqTable {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ DeqTable make_table(const float (&level)[16], float c1) {
+  uint32_t pr[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(level[2 * j], c1), __fmul_rn(level[2 * j + 1], c1));
+    pr[j] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  DeqTable t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = prmt(pr[2 * q], pr[2 * q + 1], 0x6420u);
+    t.hi[q] = prmt(pr[2 * q], pr[2 * q + 1], 0x7531u);
+  }
+  return t;
+}
+
+// 8 codes (one packed word, element j in bits 4j..4j+3) -> 4 bf16 pairs.
+__device__ __forceinline__ uint4 expand8(const DeqTable& t, uint32_t p) {
+  const uint32_t s = p & 0x77777777u;                 // low three bits of each code
+  const uint32_t x = (p >> 1) & 0x44444444u;          // bit 3 of each code, moved to bit 2
+  uint4 o;
+  {
+    const uint32_t sel = x | 0x3210u;
+    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s), prmt(t.lo[2], t.lo[3], s), sel);
+    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s), prmt(t.hi[2], t.hi[3], s), sel);
+    o.x = prmt(lo, hi, 0x5140u);
+    o.y = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t s1 = s >> 16;
+    const uint32_t sel = (x >> 16) | 0x3210u;
+    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s1), prmt(t.lo[2], t.lo[3], s1), sel);
+    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s1), prmt(t.hi[2], t.hi[3], s1), sel);
+    o.z = prmt(lo, hi, 0x5140u);
+    o.w = prmt(lo, hi, 0x7362u);
+  }
+  return o;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW>
+__global__ void __launch_bounds__(64 + 32 * NDW, 1)
+qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                  const GemmArgs args) {
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW>;
+  constexpr bool kDeq = L::kDeq;
+  constexpr bool kBMN = (BSRC == kBTmaMN || BSRC == kBDeqMN);
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(!kDeq || NDW * 32 == BN, "one dequant item per thread");
+  static_assert(NDW % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
+  constexpr uint32_t kIdesc = idesc_bf16_m128(BN, A_MN ? 1u : 0u, kBMN ? 1u : 0u);
+  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_tma = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* full_w = full_tma + NSTAGE;
+  uint64_t* empty = full_w + NSTAGE;
+  uint64_t* accum_full = empty + NSTAGE;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int c0 = blockIdx.y * BN;
+  const int split = blockIdx.z;
+  const int step_begin = split * args.steps_per_split;
+  const int step_end = min(args.k_steps, step_begin + args.steps_per_split);
+  const int n_main = max(0, step_end - step_begin);
+  const int n_lora = (split == 0) ? args.n_lora : 0;
+  const int total = n_lora + n_main;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full_tma[s], 1);
+      mbar_init(&full_w[s], NDW);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      if (n_lora > 0) { tma_prefetch_desc(&tmA2); tma_prefetch_desc(&tmB2); }
+      for (int t = 0; t < total; ++t) {
+        const int s = t % NSTAGE;
+        if (t >= NSTAGE && !mbar_wait(&empty[s], ((t / NSTAGE) - 1) & 1, abort_flag)) break;
+        uint8_t* a_dst = smem + L::kAOff + s * kATileBytes;
+        uint8_t* b_dst = smem + L::kBOff + s * L::kBTileBytes;
+        if (t < n_lora) {
+          // adapter slice: A2 = (s*U or s*V) [rows x r], K-major; B2 like the main B
+          mbar_arrive_expect_tx(&full_tma[s], kATileBytes + L::kBTileBytes);
+          tma_load_2d(a_dst, &tmA2, &full_tma[s], t * kBK, m0);
+          if (BSRC == kBDeqK || BSRC == kBTmaK) {
+            tma_load_2d(b_dst, &tmB2, &full_tma[s], t * kBK, c0);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b_dst + c * (kBK * 128), &tmB2, &full_tma[s], c0 + 64 * c, t * kBK);
+          }
+        } else {
+          const int ks = step_begin + (t - n_lora);
+          const uint32_t bbytes = kDeq ? L::kPTileBytes : L::kBTileBytes;
+          mbar_arrive_expect_tx(&full_tma[s], kATileBytes + bbytes);
+          if (A_MN) {
+            tma_load_2d(a_dst, &tmA, &full_tma[s], m0, ks * kBK);
+            tma_load_2d(a_dst + kBK * 128, &tmA, &full_tma[s], m0 + 64, ks * kBK);
+          } else {
+            tma_load_2d(a_dst, &tmA, &full_tma[s], ks * kBK, m0);
+          }
+          if (BSRC == kBTmaK) {
+            tma_load_2d(b_dst, &tmB, &full_tma[s], ks * kBK, c0);
+          } else if (BSRC == kBTmaMN) {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b_dst + c * (kBK * 128), &tmB, &full_tma[s], c0 + 64 * c, ks * kBK);
+          } else if (BSRC == kBDeqK) {
+            // packed codes of weight rows [c0, c0+BN), k-step ks: BN rows x 32 B
+            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], ks * (kBK / 2), c0);
+          } else {
+            // packed codes of weight rows [64 ks, 64 ks + 64), columns [c0, c0+BN): 64 rows x BN/2 B
+            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], c0 / 2, ks * kBK);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = true;
+    for (int t = 0; t < total && ok; ++t) {
+      const int s = t % NSTAGE;
+      const uint32_t ph = (t / NSTAGE) & 1;
+      ok = mbar_wait(&full_tma[s], ph, abort_flag);
+      if (ok && kDeq && t >= n_lora) ok = mbar_wait(&full_w[s], ph, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a_base = smem_u32(smem + L::kAOff + s * kATileBytes);
+        const uint32_t b_base = smem_u32(smem + L::kBOff + s * L::kBTileBytes);
+        // the adapter slices' A operand is always K-major
+        const bool a_mn_now = A_MN && (t >= n_lora);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = a_mn_now ? smem_desc_sw128(a_base + kk * 2048, kBK * 128)
+                                       : smem_desc_sw128(a_base + kk * 32, 16);
+          const uint64_t bd = kBMN ? smem_desc_sw128(b_base + kk * 2048, kBK * 128)
+                                   : smem_desc_sw128(b_base + kk * 32, 16);
+          umma_bf16(tmem_d, ad, bd, kIdesc, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) umma_commit(accum_full);  // also fires (immediately) when nothing was issued
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ dequant
+    const int item = threadIdx.x - 64;  // 0 .. NDW*32-1
+    bool ok = true;
+    if constexpr (kDeq) {
+      float level[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) level[i] = args.level[i];
+      // item -> (weight row, 64-block) of this thread, and where its bytes live
+      int w_row_base, kb_base, row_stride_steps;
+      if (BSRC == kBDeqK) {
+        // row `item` of the B tile = weight row c0+item, block = k-step
+        w_row_base = c0 + item;
+        kb_base = 0;
+        row_stride_steps = 0;
+      } else {
+        // item = (reduction row nr, 64-column block jb of the tile)
+        w_row_base = item & 63;           // + 64*ks
+        kb_base = c0 / 64 + (item >> 6);  // fixed block column
+        row_stride_steps = 64;
+      }
+      auto load_scale = [&](int ks) -> float {
+        const int wr = (BSRC == kBDeqK) ? w_row_base : (w_row_base + ks * row_stride_steps);
+        const int kb = (BSRC == kBDeqK) ? ks : kb_base;
+        if (wr >= args.w_rows || kb >= args.w_kblocks) return 0.f;
+        const int64_t blk = static_cast<int64_t>(wr) * args.w_kblocks + kb;
+        return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
+      };
+      float c1_next = (n_main > 0) ? load_scale(step_begin) : 0.f;
+      for (int t = n_lora; t < total; ++t) {
+        const int s = t % NSTAGE;
+        const uint32_t ph = (t / NSTAGE) & 1;
+        const int ks = step_begin + (t - n_lora);
+        const float c1 = c1_next;
+        if (t + 1 < total) c1_next = load_scale(ks + 1);
+        const DeqTable tab = make_table(level, c1);
+        if (!mbar_wait(&full_tma[s], ph, abort_flag)) { ok = false; break; }
+        const uint32_t p_base = smem_u32(smem + L::kPOff + s * L::kPTileBytes);
+        const uint32_t b_base = smem_u32(smem + L::kBOff + s * L::kBTileBytes);
+        if (BSRC == kBDeqK) {
+          // packed row `item`: 32 B, 32-byte-swizzled (16 B chunk h at h ^ ((row>>2)&1))
+          const int r = item;
+          const uint32_t sw = (r >> 2) & 1;
+          const uint4 p0 = ld_shared_v4(p_base + r * 32 + ((0u ^ sw) << 4));
+          const uint4 p1 = ld_shared_v4(p_base + r * 32 + ((1u ^ sw) << 4));
+          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          const uint32_t row_addr = b_base + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ (r & 7)) << 4), expand8(tab, words[c]));
+        } else {
+          // packed row nr: BN/2 = 128 B, 128-byte-swizzled; block jb is chunks 2jb, 2jb+1
+          const int nr = item & 63;
+          const int jb = item >> 6;
+          const uint32_t prow = p_base + nr * 128;
+          const uint4 p0 = ld_shared_v4(prow + ((static_cast<uint32_t>(2 * jb) ^ (nr & 7)) << 4));
+          const uint4 p1 = ld_shared_v4(prow + ((static_cast<uint32_t>(2 * jb + 1) ^ (nr & 7)) << 4));
+          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          const uint32_t row_addr = b_base + jb * (kBK * 128) + nr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ (nr & 7)) << 4), expand8(tab, words[c]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_w[s]);
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait(accum_full, 0, abort_flag);
+    if (ok && total > 0) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int grp = (warp - 2) >> 2;
+      const int row = m0 + q * 32 + lane;
+      for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+        tmem_ld_wait();
+        const int col = c0 + ch * 32;
+        if (row < args.m_rows && col < args.n_cols) {
+          if (OUT == kOutBf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
+                                                  static_cast<int64_t>(row) * args.ld_out + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 o;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+              o.x = *reinterpret_cast<uint32_t*>(&h0);
+              o.y = *reinterpret_cast<uint32_t*>(&h1);
+              o.z = *reinterpret_cast<uint32_t*>(&h2);
+              o.w = *reinterpret_cast<uint32_t*>(&h3);
+              dst[i] = o;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
+                                                    static_cast<int64_t>(row) * args.ld_out + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      }
+    } else if (ok && OUT == kOutF32Partial) {
+      // a split with no work still owns its slice of the partial buffer: zero it
+      const int q = warp & 3;
+      const int grp = (warp - 2) >> 2;
+      const int row = m0 + q * 32 + lane;
+      for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
+        const int col = c0 + ch * 32;
+        if (row < args.m_rows && col < args.n_cols) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
+                                                  static_cast<int64_t>(row) * args.ld_out + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Deterministic reductions of split partials (fixed split order).
+
+// U or V: P[split][M][rpad] -> plain (bf16, may be NULL) and scaled (bf16 of s*sum).
+__global__ void reduce_lora_kernel(const float* __restrict__ P, int splits, int64_t split_stride, int M,
+                                   int r, int rpad, float s, __nv_bfloat16* __restrict__ plain,
+                                   __nv_bfloat16* __restrict__ scaled) {
+  const int64_t n = static_cast<int64_t>(M) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / r;
+    const int j = static_cast<int>(i - m * r);
+    float acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += P[sp * split_stride + m * rpad + j];
+    if (plain) plain[i] = __float2bfloat16_rn(acc);
+    if (scaled) scaled[i] = __float2bfloat16_rn(s * acc);
+  }
+}
+
+// dA^T partials P[split][K][rpad] -> dA[r][K] = s * sum (transposed write);
+// dB partials Q[split][N][rpad] -> dB[N][r] = s * sum.
+__global__ void reduce_grad_kernel(const float* __restrict__ P, int splits_a, int64_t stride_a, int K,
+                                   const float* __restrict__ Q, int splits_b, int64_t stride_b, int N,
+                                   int r, int rpad, float s, float* __restrict__ dA, float* __restrict__ dB) {
+  const int64_t na = static_cast<int64_t>(r) * K;
+  const int64_t nb = static_cast<int64_t>(N) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < na + nb;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (i < na) {
+      const int64_t j = i / K;
+      const int64_t k = i - j * K;
+      float acc = 0.f;
+      for (int sp = 0; sp < splits_a; ++sp) acc += P[sp * stride_a + k * rpad + j];
+      dA[i] = s * acc;
+    } else {
+      const int64_t e = i - na;
+      const int64_t n = e / r;
+      const int64_t j = e - n * r;
+      float acc = 0.f;
+      for (int sp = 0; sp < splits_b; ++sp) acc += Q[sp * stride_b + n * rpad + j];
+      dB[e] = s * acc;
+    }
+  }
+}
+
+}  // namespace qlora

@@ -1,0 +1,587 @@
+// Host side of the C ABI declared in include/qlora_nf4.h: argument checks,
+// the NF4 tables, workspace layout, TMA descriptors and kernel launches.
+// Everything here runs on the host; all arithmetic of the layer runs in the
+// kernels of quantize.cuh and gemm_tc.cuh.
+#include "qlora_nf4.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "ptx_sm100.cuh"
+#include "quantize.cuh"
+#include "gemm_tc.cuh"
+
+using namespace qlora;
+
+namespace {
+
+// ------------------------------------------------------------------ NF4 table
+// Standard normal quantile by Newton's method on Phi(x) = erfc(-x/sqrt2)/2
+// (on the upper tail erfc(x/sqrt2)/2 = 1-p for p > 1/2), started at 0.
+double normal_quantile(double p) {
+  const double inv_sqrt_2pi = 0.39894228040143267794;
+  const bool upper = p > 0.5;
+  const double target = upper ? 1.0 - p : p;
+  double x = 0.0;
+  for (int it = 0; it < 100; ++it) {
+    const double f = upper ? (target - 0.5 * std::erfc(x / std::sqrt(2.0)))
+                           : (0.5 * std::erfc(-x / std::sqrt(2.0)) - target);
+    const double step = f / (inv_sqrt_2pi * std::exp(-0.5 * x * x));
+    const double nx = x - step;
+    if (nx == x || std::fabs(step) < 1e-17) { x = nx; break; }
+    x = nx;
+  }
+  return x;
+}
+
+// "QLoRAの理論と実装", listing create_nf4_codebook: Phi^-1(i/18) for i = 1..8,
+// the level 0, Phi^-1(j/16) for j = 9..15, divided by the largest magnitude.
+// Decision thresholds: code(n) = #{i : n > (level_i + level_{i+1})/2}, the
+// exact nearest level with the lower index on a tie; thr_i is the smallest
+// fp32 above that exact midpoint, so code(n) = #{i : n >= thr_i}.  The
+// 257-cell table indexes floor(128 n) + 128 for n in [-1, 1].
+Nf4Tables build_tables() {
+  Nf4Tables T;
+  std::memset(&T, 0, sizeof(T));
+  double v[16];
+  int n = 0;
+  for (int i = 1; i <= 8; ++i) v[n++] = normal_quantile(i / 18.0);
+  v[n++] = 0.0;
+  for (int j = 9; j <= 15; ++j) v[n++] = normal_quantile(j / 16.0);
+  double mx = 0.0;
+  for (double a : v) mx = std::max(mx, std::fabs(a));
+  for (int i = 0; i < 16; ++i) T.level[i] = static_cast<float>(v[i] / mx);
+  std::sort(T.level, T.level + 16);
+  float thr[15];
+  for (int i = 0; i < 15; ++i) {
+    const double mid = (static_cast<double>(T.level[i]) + static_cast<double>(T.level[i + 1])) * 0.5;
+    float f = static_cast<float>(mid);
+    if (static_cast<double>(f) <= mid) f = std::nextafter(f, INFINITY);
+    thr[i] = f;
+  }
+  for (int c = 0; c < kLutCells; ++c) {
+    const double lo = (c - 128) / 128.0, hi = (c - 127) / 128.0;
+    int cnt = 0;
+    float inside = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      if (thr[i] <= lo) ++cnt;
+      else if (thr[i] < hi) inside = std::min(inside, thr[i]);
+    }
+    T.cell_lo[c] = static_cast<uint8_t>(cnt);
+    T.cell_thr[c] = inside;
+  }
+  return T;
+}
+
+const Nf4Tables& tables() {
+  static const Nf4Tables t = build_tables();
+  return t;
+}
+
+// ------------------------------------------------------------------ device
+constexpr int kMaxDevices = 64;
+
+int check_device(int* dev_out, int* num_sms) {
+  static int cached_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 bad
+  static int cached_sms[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_NO_DEVICE; }
+  if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_NO_DEVICE;
+  if (cached_ok[dev] == 0) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_NO_DEVICE; }
+    cached_ok[dev] = (prop.major == 10) ? 1 : -1;
+    cached_sms[dev] = prop.multiProcessorCount;
+  }
+  if (cached_ok[dev] != 1) return QLORA_ERR_NO_DEVICE;
+  *dev_out = dev;
+  *num_sms = cached_sms[dev];
+  return QLORA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ TMA
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor: `cols` contiguous elements per row, `rows` rows,
+// `row_bytes` between rows; box of box_cols x box_rows.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, cols * 2, box_cols, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// ------------------------------------------------------------------ timing
+struct TimingRec {
+  int kind;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+bool g_timing_on = false;
+std::vector<TimingRec> g_timing_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) { cudaGetLastError(); return nullptr; }
+  return e;
+}
+
+// Run `launch` (which enqueues one kernel on st); bracket it with events when
+// timing is on.
+template <class F>
+int timed(int kind, cudaStream_t st, F&& launch) {
+  if (!g_timing_on) return launch();
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  cudaEvent_t a = take_event(), b = take_event();
+  if (a) cudaEventRecord(a, st);
+  const int rc = launch();
+  if (b) cudaEventRecord(b, st);
+  if (a && b) g_timing_recs.push_back({kind, a, b});
+  return rc;
+}
+
+// ------------------------------------------------------------------ launches
+template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW>
+int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW>;
+  auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW>;
+  static bool attr_set[kMaxDevices];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const int kind = (BSRC == kBDeqK) ? QLORA_KERNEL_FWD
+                 : (BSRC == kBDeqMN) ? QLORA_KERNEL_DX
+                 : A_MN ? QLORA_KERNEL_GRAD_GEMM : QLORA_KERNEL_LORA_GEMM;
+  return timed(kind, st, [&] {
+    kern<<<grid, 64 + 32 * NDW, L::kDynBytes, st>>>(a, b, a2, b2, args);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  });
+}
+
+struct SplitPlan {
+  int tiles_m, tiles_n, k_steps, splits, per_split;
+};
+
+SplitPlan plan_split(int64_t rows, int64_t cols_pad, int64_t k_steps, int bn, int num_sms) {
+  SplitPlan p;
+  p.tiles_m = static_cast<int>((rows + kBM - 1) / kBM);
+  p.tiles_n = static_cast<int>(cols_pad / bn);
+  p.k_steps = static_cast<int>(k_steps);
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int target = 2 * num_sms;
+  int splits = std::max(1, std::min<int>(p.k_steps, (target + tiles - 1) / tiles));
+  p.per_split = (p.k_steps + splits - 1) / splits;
+  p.splits = (p.k_steps + p.per_split - 1) / p.per_split;
+  return p;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t us, v, vs, u, part, total;
+  SplitPlan pu, pv, pa, pb;
+};
+
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+  WsLayout w;
+  const int64_t rpad = (r + 63) / 64 * 64;
+  w.pu = plan_split(M, rpad, K / 64, 64, num_sms);
+  w.pv = plan_split(M, rpad, N / 64, 64, num_sms);
+  w.pa = plan_split(K, rpad, (M + 63) / 64, 64, num_sms);
+  w.pb = plan_split(N, rpad, (M + 63) / 64, 64, num_sms);
+  const size_t mr = a256(static_cast<size_t>(M) * r * 2);
+  const size_t part_u = static_cast<size_t>(w.pu.splits) * M * rpad;
+  const size_t part_v = static_cast<size_t>(w.pv.splits) * M * rpad;
+  const size_t part_ab = static_cast<size_t>(w.pa.splits) * K * rpad + a256(static_cast<size_t>(w.pb.splits) * N * rpad * 4) / 4;
+  const size_t part = std::max(part_u, std::max(part_v, part_ab)) * 4;
+  w.us = 0;
+  w.v = w.us + mr;
+  w.vs = w.v + mr;
+  w.u = w.vs + mr;
+  w.part = w.u + mr;
+  w.total = w.part + a256(part);
+  return w;
+}
+
+int check_weight(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K) {
+  if (!codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || K % 64 != 0 || N % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (N > (1 << 24) || K > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes) || !aligned16(s2)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+int check_lora(const void* X, int64_t M, const void* A, const void* B, int r, float alpha) {
+  if (!X || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (M < 1 || M > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (r % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+void fill_levels(GemmArgs& g) {
+  for (int i = 0; i < 16; ++i) g.level[i] = tables().level[i];
+}
+
+// U = X A^T into `plain` (bf16, may be NULL) and `scaled` = bf16(s U) (may be NULL).
+int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat, int r, float s,
+                  uint16_t* plain, uint16_t* scaled, float* part, const SplitPlan& p, cudaStream_t st,
+                  int dev) {
+  const int rpad = (r + 63) / 64 * 64;
+  CUtensorMap ta, tb;
+  if (!map_bf16(&ta, X, M, K, 64, 128) || !map_bf16(&tb, Amat, r, K, 64, 64)) return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.m_rows = static_cast<int>(M);
+  g.n_cols = rpad;
+  g.k_steps = p.k_steps;
+  g.steps_per_split = p.per_split;
+  g.n_lora = 0;
+  g.out = part;
+  g.ld_out = rpad;
+  g.split_stride = M * rpad;
+  int rc = launch_gemm<64, 4, false, kBTmaK, kOutF32Partial, 4>(dim3(p.tiles_m, p.tiles_n, p.splits), ta, tb, ta,
+                                                                tb, g, st, dev);
+  if (rc) return rc;
+  const int64_t n = M * r;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  return timed(QLORA_KERNEL_LORA_REDUCE, st, [&] {
+    reduce_lora_kernel<<<blocks, 256, 0, st>>>(part, p.splits, M * rpad, static_cast<int>(M), r, rpad, s,
+                                               reinterpret_cast<__nv_bfloat16*>(plain),
+                                               reinterpret_cast<__nv_bfloat16*>(scaled));
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  });
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+const char* qlora_strerror(int code) {
+  switch (code) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument (NULL pointer, r or alpha out of range)";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or alignment (K, N multiple of 64; r multiple of 8; 16-byte aligned pointers)";
+    case QLORA_ERR_CUDA: return "CUDA runtime error";
+    case QLORA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown error code";
+  }
+}
+
+int qlora_nf4_codebook(float* out) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(out, tables().level, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, uint8_t* q8, float* s2,
+                          void* stream) {
+  if (!W || !codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
+  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(s2) & 3u))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const int64_t n_blocks = n_out * k_in / kBlock;
+  const int64_t groups = (n_blocks + kGroup - 1) / kGroup;
+  if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
+    quantize_dq_kernel<<<static_cast<unsigned>(groups), 256, 0, st>>>(W, n_blocks, codes, q8, s2, tables());
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  });
+}
+
+int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                  void* out, int out_dtype, void* stream) {
+  if (!codes || !q8 || !s2 || !out) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != QLORA_OUT_BF16 && out_dtype != QLORA_OUT_FP32) return QLORA_ERR_INVALID_ARG;
+  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const int64_t n_oct = n_out * k_in / 8;
+  const int blocks = static_cast<int>(std::min<int64_t>((n_oct + 255) / 256, 64LL * sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return timed(QLORA_KERNEL_DEQUANT, st, [&] {
+    if (out_dtype == QLORA_OUT_BF16)
+      dequant_kernel<true><<<blocks, 256, 0, st>>>(codes, q8, s2, n_oct, out, tables());
+    else
+      dequant_kernel<false><<<blocks, 256, 0, st>>>(codes, q8, s2, n_oct, out, tables());
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  });
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 1 || n_out < 64 || k_in < 64 || r < 1 || r > 256) return 0;
+  int dev = 0, sms = 148;
+  if (check_device(&dev, &sms) != QLORA_OK) sms = 148;
+  return ws_layout(M, n_out, k_in, r, sms).total;
+}
+
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* Y, uint16_t* U_save, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
+  if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
+  if (!Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const WsLayout L = ws_layout(M, n_out, k_in, r, sms);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* Us = reinterpret_cast<uint16_t*>(ws + L.us);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  const float s = alpha / static_cast<float>(r);
+  const int rpad = (r + 63) / 64 * 64;
+
+  if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, part, L.pu, st, dev)) return rc;
+
+  CUtensorMap tx, tp, tus, tb;
+  if (!map_bf16(&tx, X, M, k_in, 64, 128) ||
+      !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 256,
+                CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 256))
+    return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.m_rows = static_cast<int>(M);
+  g.n_cols = static_cast<int>(n_out);
+  g.k_steps = static_cast<int>(k_in / 64);
+  g.steps_per_split = g.k_steps;
+  g.n_lora = rpad / 64;
+  g.q8 = q8;
+  g.s2 = s2;
+  g.w_rows = static_cast<int>(n_out);
+  g.w_kblocks = static_cast<int>(k_in / 64);
+  fill_levels(g);
+  g.out = Y;
+  g.ld_out = n_out;
+  g.split_stride = 0;
+  const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256), 1);
+  return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8>(grid, tx, tp, tus, tb, g, st, dev);
+}
+
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     const uint16_t* dY, const uint16_t* U_saved, uint16_t* dX, float* dA, float* dB,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
+  if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
+  if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (U_saved && !aligned16(U_saved)) ||
+      (dX && !aligned16(dX)))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const WsLayout L = ws_layout(M, n_out, k_in, r, sms);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* V = reinterpret_cast<uint16_t*>(ws + L.v);
+  uint16_t* Vs = reinterpret_cast<uint16_t*>(ws + L.vs);
+  uint16_t* Ubuf = reinterpret_cast<uint16_t*>(ws + L.u);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  const float s = alpha / static_cast<float>(r);
+  const int rpad = (r + 63) / 64 * 64;
+  const int N = static_cast<int>(n_out), K = static_cast<int>(k_in);
+
+  // V = dY B  (B viewed MN-major: its rows are the reduction index)
+  {
+    CUtensorMap ta, tb;
+    if (!map_bf16(&ta, dY, M, N, 64, 128) || !map_bf16(&tb, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.m_rows = static_cast<int>(M);
+    g.n_cols = rpad;
+    g.k_steps = L.pv.k_steps;
+    g.steps_per_split = L.pv.per_split;
+    g.out = part;
+    g.ld_out = rpad;
+    g.split_stride = M * rpad;
+    if (int rc = launch_gemm<64, 4, false, kBTmaMN, kOutF32Partial, 4>(dim3(L.pv.tiles_m, L.pv.tiles_n, L.pv.splits),
+                                                                      ta, tb, ta, tb, g, st, dev))
+      return rc;
+    const int64_t n = M * r;
+    if (int rc = timed(QLORA_KERNEL_LORA_REDUCE, st, [&] {
+          reduce_lora_kernel<<<static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)), 256, 0, st>>>(
+              part, L.pv.splits, M * rpad, static_cast<int>(M), r, rpad, s, reinterpret_cast<__nv_bfloat16*>(V),
+              reinterpret_cast<__nv_bfloat16*>(Vs));
+          return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+        }))
+      return rc;
+  }
+  // U (from the forward, or recomputed)
+  const uint16_t* U = U_saved;
+  if (!U) {
+    if (int rc = run_lora_down(X, M, K, A, r, s, Ubuf, nullptr, part, L.pu, st, dev)) return rc;
+    U = Ubuf;
+  }
+  // dX = dY dequant(W) + (s V) A
+  if (dX) {
+    CUtensorMap ta, tp, ta2, tb2;
+    if (!map_bf16(&ta, dY, M, N, 64, 128) ||
+        !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
+      return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.m_rows = static_cast<int>(M);
+    g.n_cols = K;
+    g.k_steps = N / 64;
+    g.steps_per_split = g.k_steps;
+    g.n_lora = rpad / 64;
+    g.q8 = q8;
+    g.s2 = s2;
+    g.w_rows = N;
+    g.w_kblocks = K / 64;
+    fill_levels(g);
+    g.out = dX;
+    g.ld_out = K;
+    const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256), 1);
+    if (int rc = launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8>(grid, ta, tp, ta2, tb2, g, st, dev)) return rc;
+  }
+  // dA^T = X^T V and dB = dY^T U, reduced over M in split partials
+  float* part_a = part;
+  float* part_b = part + static_cast<size_t>(L.pa.splits) * K * rpad;
+  {
+    CUtensorMap ta, tb;
+    if (!map_bf16(&ta, X, M, K, 64, 64) || !map_bf16(&tb, V, M, r, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.m_rows = K;
+    g.n_cols = rpad;
+    g.k_steps = L.pa.k_steps;
+    g.steps_per_split = L.pa.per_split;
+    g.out = part_a;
+    g.ld_out = rpad;
+    g.split_stride = static_cast<int64_t>(K) * rpad;
+    if (int rc = launch_gemm<64, 4, true, kBTmaMN, kOutF32Partial, 4>(dim3(L.pa.tiles_m, L.pa.tiles_n, L.pa.splits),
+                                                                     ta, tb, ta, tb, g, st, dev))
+      return rc;
+  }
+  {
+    CUtensorMap ta, tb;
+    if (!map_bf16(&ta, dY, M, N, 64, 64) || !map_bf16(&tb, U, M, r, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.m_rows = N;
+    g.n_cols = rpad;
+    g.k_steps = L.pb.k_steps;
+    g.steps_per_split = L.pb.per_split;
+    g.out = part_b;
+    g.ld_out = rpad;
+    g.split_stride = static_cast<int64_t>(N) * rpad;
+    if (int rc = launch_gemm<64, 4, true, kBTmaMN, kOutF32Partial, 4>(dim3(L.pb.tiles_m, L.pb.tiles_n, L.pb.splits),
+                                                                     ta, tb, ta, tb, g, st, dev))
+      return rc;
+  }
+  {
+    const int64_t n = static_cast<int64_t>(r) * K + static_cast<int64_t>(N) * r;
+    if (int rc = timed(QLORA_KERNEL_GRAD_REDUCE, st, [&] {
+          reduce_grad_kernel<<<static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)), 256, 0, st>>>(
+              part_a, L.pa.splits, static_cast<int64_t>(K) * rpad, K, part_b, L.pb.splits,
+              static_cast<int64_t>(N) * rpad, N, r, rpad, s, dA, dB);
+          return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+        }))
+      return rc;
+  }
+  return QLORA_OK;
+}
+
+int qlora_timing_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  for (auto& r : g_timing_recs) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_timing_recs.clear();
+  g_timing_on = on != 0;
+  return QLORA_OK;
+}
+
+int qlora_timing_collect(double* ms, int64_t* counts, int n_kinds) {
+  if (!ms || !counts || n_kinds < QLORA_KERNEL_COUNT) return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  int rc = QLORA_OK;
+  for (auto& r : g_timing_recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
+      cudaGetLastError();
+      rc = QLORA_ERR_CUDA;
+    } else {
+      ms[r.kind] += t;
+      counts[r.kind] += 1;
+    }
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_timing_recs.clear();
+  return rc;
+}
+
+int qlora_device_status(void* stream) {
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (flag) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_ERR_DEVICE_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+// NF4 quantization with double quantization, and dequantization, for sm_100a.
+//
+// "QLoRAの理論と実装" §5-1 (absmax per 64-block, w/absmax, nearest of the 16
+// NormalFloat levels, 4-bit code) and §5-2 (8-bit re-quantization of the fp32
+// absmax constants in groups of 256, one fp32 second-level constant).
+//
+// quantize_dq_kernel: one CTA per group of 256 blocks (16384 weights, 64 KiB
+// of fp32 input).  Eight threads share a 64-block (8 consecutive weights each,
+// two 16-byte loads), so a warp reads 1 KiB contiguous per pass; the block
+// absmax is a 3-step xor-shuffle max.  The nearest level comes from a
+// 257-cell lookup table over floor(128 * w_norm) (every cell of width 1/128
+// holds at most one decision threshold), so the search is one shared-memory
+// load and one compare.  The group's 256 absmax values then stay in shared
+// memory for the second-level quantization, so the fp32 constants never go to
+// HBM.  Traffic per weight: 4 B read, 0.5 + 1/64 + 4/16384 B written.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace qlora {
+
+constexpr int kBlock = 64;     // first-level block
+constexpr int kGroup = 256;    // second-level group (blocks per s2)
+constexpr int kLutCells = 257; // floor(128 n) + 128 for n in [-1, 1]
+
+// Host-built tables handed to the kernels by value.
+struct Nf4Tables {
+  float level[16];             // NF4 levels, ascending (fp32)
+  float cell_thr[kLutCells];   // the decision threshold inside the cell, or +inf
+  uint8_t cell_lo[kLutCells];  // code of the cell's left edge
+};
+
+__global__ void __launch_bounds__(256)
+quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
+                   uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
+  __shared__ float s_thr[kLutCells];
+  __shared__ int s_lo[kLutCells];
+  __shared__ float s_absmax[kGroup];
+  __shared__ float s_warpmax[8];
+
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kLutCells; i += blockDim.x) {
+    s_thr[i] = tabs.cell_thr[i];
+    s_lo[i] = tabs.cell_lo[i];
+  }
+
+  const int64_t g = blockIdx.x;
+  const int64_t b_first = g * kGroup;
+  const int64_t left = n_blocks - b_first;
+  const int nb = left < kGroup ? static_cast<int>(left) : kGroup;
+  const int sub = tid & 7;     // 8 threads per 64-block
+  const int lb0 = tid >> 3;    // block within a pass (32 blocks per pass)
+
+  // Issue every load of the group up front (16 x 16 B per thread in flight).
+  float4 v[8][2];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int lb = p * 32 + lb0;
+    if (lb < nb) {
+      const float4* src = reinterpret_cast<const float4*>(W + (b_first + lb) * kBlock + sub * 8);
+      v[p][0] = __ldcs(src);
+      v[p][1] = __ldcs(src + 1);
+    } else {
+      v[p][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      v[p][1] = v[p][0];
+    }
+  }
+  __syncthreads();  // lookup table ready
+
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int lb = p * 32 + lb0;
+    float e[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
+                  v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
+    float am = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(e[j]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+    if (lb < nb) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // one IEEE fp32 division, round to nearest (never the reciprocal form)
+        const float wn = am > 0.f ? __fdiv_rn(e[j], am) : 0.f;
+        int cell = __float2int_rd(wn * 128.f) + 128;   // exact: scaling by 2^7
+        cell = min(max(cell, 0), kLutCells - 1);
+        const int code = s_lo[cell] + (wn >= s_thr[cell] ? 1 : 0);
+        packed |= static_cast<uint32_t>(code) << (4 * j);
+      }
+      *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
+      if (sub == 0) s_absmax[lb] = am;
+    }
+  }
+  __syncthreads();
+
+  // Second level: c2 = max of the group's absmax, s2 = fp32(c2/255),
+  // q = min(255, rint_half_even(fp32(absmax/s2))).
+  const float my = tid < nb ? s_absmax[tid] : 0.f;
+  float m = my;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((tid & 31) == 0) s_warpmax[tid >> 5] = m;
+  __syncthreads();
+  float c2 = s_warpmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_warpmax[w]);
+  const float sc = __fdiv_rn(c2, 255.f);
+  if (tid < nb) {
+    int q = 0;
+    if (sc != 0.f) {
+      const float ratio = __fdiv_rn(my, sc);
+      q = min(255, __float2int_rn(ratio));  // round half to even
+    }
+    q8[b_first + tid] = static_cast<uint8_t>(q);
+  }
+  if (tid == 0) s2[g] = sc;
+}
+
+// Dense dequantization: w = fp32(level[code] * fp32(q * s2)), fp32 or bf16 out.
+// One thread per 8 consecutive weights (4 packed bytes).
+template <bool kBf16>
+__global__ void __launch_bounds__(256)
+dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8,
+               const float* __restrict__ s2, int64_t n_oct, void* __restrict__ out,
+               const Nf4Tables tabs) {
+  __shared__ float s_level[16];
+  if (threadIdx.x < 16) s_level[threadIdx.x] = tabs.level[threadIdx.x];
+  __syncthreads();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_oct;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(codes) + i);
+    const int64_t blk = (i * 8) / kBlock;
+    const float c1 = __fmul_rn(static_cast<float>(__ldg(q8 + blk)), __ldg(s2 + blk / kGroup));
+    float w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(s_level[(p >> (4 * j)) & 15u], c1);
+    if (kBf16) {
+      uint4 o;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(w[0], w[1]);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(w[2], w[3]);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(w[4], w[5]);
+      __nv_bfloat162 h3 = __floats2bfloat162_rn(w[6], w[7]);
+      o.x = *reinterpret_cast<uint32_t*>(&h0);
+      o.y = *reinterpret_cast<uint32_t*>(&h1);
+      o.z = *reinterpret_cast<uint32_t*>(&h2);
+      o.w = *reinterpret_cast<uint32_t*>(&h3);
+      reinterpret_cast<uint4*>(out)[i] = o;
+    } else {
+      float4* o = reinterpret_cast<float4*>(out) + 2 * i;
+      o[0] = make_float4(w[0], w[1], w[2], w[3]);
+      o[1] = make_float4(w[4], w[5], w[6], w[7]);
+    }
+  }
+}
+
+}  // namespace qlora

@@ -1,0 +1,185 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA NF4 linear-layer library.
+ *
+ * The library implements the data-parallel hot path of QLoRA (Dettmers et al.
+ * 2023) as described on the pages "QLoRAの理論と実装" (disassemble-channel.com)
+ * and the Qiita article on why QLoRA survives 4-bit:
+ *
+ *   1. blockwise NF4 quantization of a frozen fp32 weight with double
+ *      quantization of its absmax constants (§5-1 and §5-2 of the first page);
+ *   2. the frozen-NF4 linear layer with its LoRA adapter, computed in bf16
+ *      (the "storage 4-bit / compute BF16" split), forward and backward
+ *      ("QLoRAの計算フロー", "逆伝播と勾配の流れ").
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Shapes: the weight W is N x K (n_out x k_in), row-major, the pages' d x k.
+ *   Activations X are M x K (tokens x in), outputs Y are M x N.  LoRA A is
+ *   r x K, B is N x r, the adapter scale is s = alpha / r.
+ * - bf16 tensors are passed as uint16_t bit patterns; fp32 as float.
+ * - Every pointer argument is a DEVICE pointer (CUDA global memory on the
+ *   current device), except where a comment says "host".  The caller owns
+ *   every buffer; the library allocates no device memory.  Scratch comes from
+ *   the caller's `workspace` (size from qlora_workspace_bytes).
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call is asynchronous on that stream: it validates its arguments on
+ *   the host, enqueues kernels and returns.
+ * - The quantized weight is three flat buffers:
+ *     codes  uint8_t[N*K/2]      NF4 codes, row-major, element 2j in the low
+ *                                nibble of byte j;
+ *     q8     uint8_t[N*K/64]     8-bit absmax constant of each 64-block;
+ *     s2     float[ceil(N*K/16384)]  fp32 second-level constant of each group
+ *                                of 256 consecutive blocks.
+ *   Fixed by the method: block 64, group 256, double quantization on.
+ * - Preconditions checked on the host (QLORA_ERR_* on violation, nothing
+ *   enqueued): non-NULL required pointers, every pointer 16-byte aligned,
+ *   K % 64 == 0, N % 64 == 0, M >= 1, 1 <= r <= 256 with r % 8 == 0, alpha
+ *   finite.  NaN or Inf inside W is a caller error; the result is unspecified.
+ * - Return value: QLORA_OK (0) or a negative QLORA_ERR_* code.  Errors raised
+ *   on the device after a call returned (a bounded wait inside a kernel that
+ *   gave up) are latched in a device flag and reported by qlora_device_status.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QLORA_OK 0
+#define QLORA_ERR_INVALID_ARG (-1)     /* NULL pointer, r or alpha out of range    */
+#define QLORA_ERR_UNSUPPORTED_SHAPE (-2) /* K or N not a multiple of 64, misalignment */
+#define QLORA_ERR_CUDA (-3)            /* a CUDA runtime call or launch failed      */
+#define QLORA_ERR_DEVICE_TIMEOUT (-4)  /* a kernel's bounded wait expired           */
+#define QLORA_ERR_WORKSPACE (-5)       /* workspace NULL or smaller than required   */
+#define QLORA_ERR_NO_DEVICE (-6)       /* no sm_100 device is current               */
+
+#define QLORA_OUT_BF16 0
+#define QLORA_OUT_FP32 1
+
+/* Human-readable name of a return code (static string, never NULL). */
+const char* qlora_strerror(int code);
+
+/*
+ * The 16 NF4 levels, ascending, as fp32 (host pointer `out`, 16 floats).
+ * Built once on the host from the quantile definition of "QLoRAの理論と実装",
+ * listing create_nf4_codebook (levels Phi^-1(i/18), i=1..8, then 0, then
+ * Phi^-1(j/16), j=9..15, divided by |Phi^-1(1/18)|).  Returns QLORA_OK.
+ */
+int qlora_nf4_codebook(float* out);
+
+/*
+ * Blockwise NF4 quantization with double quantization.
+ * "QLoRAの理論と実装" §5-1 (steps 1-2: absmax per 64 elements, w/absmax,
+ * nearest of the 16 levels stored in 4 bits) and §5-2 (the fp32 absmax
+ * constants re-quantized to 8 bits in groups of 256 with one fp32
+ * second-level constant); the Qiita page's W ~ (c2 * c1_quant) * W_quant.
+ *
+ *   W      fp32[N*K] device, row-major, read only.
+ *   codes  uint8_t[N*K/2]   written.
+ *   q8     uint8_t[N*K/64]  written.
+ *   s2     float[ceil(N*K/16384)] written.
+ * Per block: absmax = max|w|; n = fp32(w/absmax) (0 if absmax == 0); code =
+ * exact nearest level, lowest index on a tie.  Per group of 256 blocks:
+ * s2 = fp32(max absmax / 255); q = min(255, round-half-even(fp32(absmax/s2))),
+ * q = 0 when s2 == 0.  One kernel launch.
+ */
+int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in,
+                          uint8_t* codes, uint8_t* q8, float* s2, void* stream);
+
+/*
+ * Dequantization to a dense N x K matrix ("QLoRAの理論と実装" §5-1 step 3 with
+ * the two-level constant):  w = fp32(level[code] * fp32(q8 * s2)), written as
+ * fp32 (out_dtype QLORA_OUT_FP32) or rounded to nearest-even bf16
+ * (QLORA_OUT_BF16).  `out` is device memory of N*K elements.  This is for
+ * tests and export; the linear layer never materialises it.
+ */
+int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                  int64_t n_out, int64_t k_in, void* out, int out_dtype,
+                  void* stream);
+
+/* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd need for these sizes
+ * (0 on invalid sizes).  The workspace is device memory, 256-byte aligned,
+ * owned by the caller; its contents need not be initialised and are not
+ * preserved between calls. */
+size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r);
+
+/*
+ * Forward of the frozen-NF4 linear layer with LoRA, "QLoRAの計算フロー"
+ * steps 1-4 and "LoRAの復習" (h = W0 x + (alpha/r) B A x), row-major:
+ *
+ *   U = X A^T                        (M x r, fp32 accumulate)
+ *   Y = X dequant(W)^T + s U B^T     (M x N, fp32 accumulate, bf16 out)
+ *
+ * dequant(W) is rebuilt tile by tile in shared memory and consumed there by
+ * the tensor cores; no dense copy of W is written.
+ *   X  bf16[M*K], A bf16[r*K], B bf16[N*r]  read.
+ *   Y  bf16[M*N]  written.
+ *   U_save bf16[M*r] written with U (for the backward pass) unless NULL.
+ */
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                     int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M,
+                     const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* Y, uint16_t* U_save,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward, "逆伝播と勾配の流れ" (W frozen, gradients reach A and B only):
+ *
+ *   V  = dY B                                  (M x r)
+ *   dB = s dY^T U        (dL/dB = (alpha/r) dL/dY (A X)^T)     fp32 N x r
+ *   dA = s V^T X         (dL/dA = (alpha/r) B^T dL/dY X^T)     fp32 r x K
+ *   dX = dY dequant(W) + s V A   (chain rule through both paths) bf16 M x K
+ *
+ *   dY bf16[M*N] read; U_saved bf16[M*r] from the forward, or NULL to
+ *   recompute U = X A^T here.  dX may be NULL (not computed).  dA and dB are
+ *   overwritten (not accumulated).  The reductions over M are deterministic:
+ *   the same inputs give bit-identical dA and dB on every call.
+ */
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                     int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M,
+                     const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     const uint16_t* dY, const uint16_t* U_saved,
+                     uint16_t* dX, float* dA, float* dB,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error flag of the
+ * current device: QLORA_OK, QLORA_ERR_DEVICE_TIMEOUT if a kernel's bounded
+ * wait expired since the last call, or QLORA_ERR_CUDA if the stream reports a
+ * CUDA error.
+ */
+int qlora_device_status(void* stream);
+
+/*
+ * Launch timing (measurement support; no counterpart on the pages).
+ * While enabled, the library records a CUDA event pair on the launching
+ * stream around every kernel it enqueues.  qlora_timing_collect synchronises
+ * those events, adds each launch's elapsed milliseconds to ms[kind] and
+ * counts[kind] (host arrays of QLORA_KERNEL_COUNT entries, accumulated into,
+ * not overwritten) and forgets them.  Kinds are the QLORA_KERNEL_* values.
+ * Enabling clears any uncollected records.  Not thread-safe with respect to
+ * concurrent calls from several host threads while enabled.
+ */
+#define QLORA_KERNEL_QUANTIZE 0    /* NF4 + double quant                     */
+#define QLORA_KERNEL_DEQUANT 1     /* dense dequantization                   */
+#define QLORA_KERNEL_LORA_GEMM 2   /* U = X A^T or V = dY B (split partials)  */
+#define QLORA_KERNEL_LORA_REDUCE 3 /* reduction of U / V partials            */
+#define QLORA_KERNEL_FWD 4         /* fused dequant GEMM: Y                   */
+#define QLORA_KERNEL_DX 5          /* fused transposed-dequant GEMM: dX       */
+#define QLORA_KERNEL_GRAD_GEMM 6   /* dA^T = X^T V, dB = dY^T U (partials)    */
+#define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
+#define QLORA_KERNEL_COUNT 8
+int qlora_timing_enable(int on);
+int qlora_timing_collect(double* ms, int64_t* counts, int n_kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,111 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, builds the same NF4 table as the oracle, and rejects bad
+arguments on the host (no GPU is touched: validation precedes any CUDA call).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import bit_nf4_quantized_quantize_b200 as q
+from bit_nf4_quantized_quantize_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return q.load()
+
+
+def header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(qlora_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = header_functions()
+    assert {"qlora_quantize_nf4_dq", "qlora_dequant", "qlora_linear_fwd", "qlora_linear_bwd"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared <= q.exported_symbols() | declared  # binding covers the header
+    assert declared == set(q._binding._SIGNATURES)
+
+
+def test_library_codebook_equals_oracle_bitwise(lib):
+    ours = q.qlora_nf4_codebook()
+    _, ref = oracle.nf4_codebook()
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+def test_strerror(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -99):
+        assert isinstance(q.qlora_strerror(code), str) and q.qlora_strerror(code)
+
+
+def test_workspace_bytes(lib):
+    assert q.qlora_workspace_bytes(16, 256, 256, 8) > 0
+    assert q.qlora_workspace_bytes(4096, 4096, 4096, 64) > 4096 * 64 * 2
+    assert q.qlora_workspace_bytes(0, 256, 256, 8) == 0
+    assert q.qlora_workspace_bytes(16, 256, 256, 0) == 0
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_host_validation_without_gpu(lib):
+    P = 1 << 20  # a fake, 16-byte-aligned address: validation fails before any use
+    null = None
+    # quantize: null pointers, bad K
+    assert lib.qlora_quantize_nf4_dq(null, 64, 64, _p(P), _p(P), _p(P), null) == -1
+    assert lib.qlora_quantize_nf4_dq(_p(P), 64, 63, _p(P), _p(P), _p(P), null) == -2
+    assert lib.qlora_quantize_nf4_dq(_p(P + 4), 64, 64, _p(P), _p(P), _p(P), null) == -2
+    # dequant: bad dtype
+    assert lib.qlora_dequant(_p(P), _p(P), _p(P), 64, 64, _p(P), 7, null) == -1
+    args = dict(N=256, K=256, M=16, r=8, alpha=16.0)
+
+    def fwd(codes=P, X=P, M=16, r=8, alpha=16.0, N=256, K=256, Y=P, ws=P, wsb=1 << 30):
+        return lib.qlora_linear_fwd(_p(codes) if codes else null, _p(P), _p(P), N, K, _p(X) if X else null, M,
+                                    _p(P), _p(P), r, alpha, _p(Y) if Y else null, null, _p(ws) if ws else null,
+                                    wsb, null)
+
+    assert fwd(codes=0) == -1
+    assert fwd(X=0) == -1
+    assert fwd(Y=0) == -1
+    assert fwd(K=100) == -2
+    assert fwd(N=100) == -2
+    assert fwd(M=0) == -2
+    assert fwd(r=0) == -1
+    assert fwd(r=300) == -1
+    assert fwd(r=12) == -2
+    assert fwd(alpha=float("nan")) == -1
+    assert fwd(X=P + 8) == -2
+    # everything valid: the first CUDA query fails on a machine without a B200
+    rc = fwd()
+    assert rc in (-6, -5, 0) or rc == -3
+
+    def bwd(dY=P, dA=P, dB=P):
+        return lib.qlora_linear_bwd(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                    _p(dY) if dY else null, null, null, _p(dA) if dA else null,
+                                    _p(dB) if dB else null, _p(P), 1 << 30, null)
+
+    assert bwd(dY=0) == -1
+    assert bwd(dA=0) == -1
+    assert bwd(dB=0) == -1
+    assert bwd(dY=P + 2) == -2
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        q.qlora_quantize_nf4_dq(torch.zeros(64, 64))

@@ -1,0 +1,109 @@
+"""Linear layer forward/backward on the GPU against the fp64 oracle.
+
+The oracle quantizes W itself (its codes are independently checked to be
+identical to the GPU's), dequantizes to bf16 and evaluates the layer in fp64 on
+the exact bf16 operands.  Tolerance: relative L2 <= 4e-3 on every output and
+gradient.  Cases span several tiles with ragged tails in M, N and K, adapter
+ranks from 8 to 256 (one to four adapter slices), the tiny and decode
+workloads in full, and the 4096^3 training workload on sampled rows (dA, dB in
+full).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import bit_nf4_quantized_quantize_b200 as q
+from bit_nf4_quantized_quantize_b200 import synth
+from common import REL_L2_TOL, bf16_to_np_f64, bits_f64, oracle_weight, rel_l2, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(inp, rows=None, check_bwd=True, dy_rows=None):
+    N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
+    Wd = torch.from_numpy(inp["W"]).cuda()
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(Wd)
+    X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
+    U = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    Y = q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, U_save=U)
+    res = {"Y": Y, "U": U}
+    if check_bwd:
+        dX, dA, dB = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U)
+        res.update(dX=dX, dA=dA, dB=dB)
+    assert q.qlora_device_status() == 0
+    # oracle on the same inputs
+    _, _, _, What = oracle_weight(inp["W"])
+    Xo, Ao, Bo, dYo = (bits_f64(inp[k]) for k in ("X", "A", "B", "dY"))
+    Yr, Ur = oracle.linear_fwd(Xo, What, Ao, Bo, alpha, rows=rows)
+    sel = slice(None) if rows is None else rows
+    errs = {"Y": rel_l2(bf16_to_np_f64(Y)[sel], Yr), "U": rel_l2(bf16_to_np_f64(U)[sel], Ur)}
+    if check_bwd:
+        dXr, dAr, dBr = oracle.linear_bwd(Xo, What, Ao, Bo, dYo, alpha, rows=rows)
+        errs["dX"] = rel_l2(bf16_to_np_f64(res["dX"])[sel], dXr)
+        errs["dA"] = rel_l2(res["dA"].cpu().numpy(), dAr)
+        errs["dB"] = rel_l2(res["dB"].cpu().numpy(), dBr)
+    for k, e in errs.items():
+        assert e <= REL_L2_TOL, (k, e, errs)
+    return res, errs
+
+
+def test_tiny_workload_fwd_bwd():
+    run_case(synth.layer_inputs("tiny"))
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (300, 512, 768, 16),     # ragged M (2 full tiles + 44), several N and K tiles
+    (1, 256, 256, 8),        # a single token
+    (7, 320, 320, 8),        # ragged N and K tiles (320 = 256 + 64)
+    (129, 384, 640, 64),     # one row past a tile; N, K not multiples of 256
+    (200, 256, 512, 128),    # two adapter slices
+    (64, 512, 256, 256),     # four adapter slices
+    (513, 1024, 1152, 24),   # rank not a multiple of 16
+])
+def test_shapes_and_ranks(M, N, K, r):
+    run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=100 + M))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_workload_forward(M):
+    run_case(synth.layer_inputs("decode", M=M), check_bwd=False)
+
+
+def test_train4096_sampled_rows():
+    inp = synth.layer_inputs("train4096")
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 67), [0, 127, 128, 4095]]))
+    run_case(inp, rows=rows)
+
+
+def test_llama7b_down_proj_sampled_rows():
+    """The 7B stack's down projection (4096 x 11008, outlier weights), M = 2048."""
+    inp = synth.layer_inputs("llama7b", layer=6)
+    rows = np.arange(0, 2048, 97)
+    run_case(inp, rows=rows)
+
+
+def test_gradients_deterministic_and_recompute_path():
+    inp = synth.layer_inputs("tiny", M=333, shape=(512, 512), r=32, seed=77)
+    N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
+    U = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, U_save=U)
+    r1 = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U)
+    r2 = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U)
+    r3 = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=None)
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+    for a, b in zip(r1, r3):
+        assert torch.equal(a, b)
+    _, dA4, dB4 = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U, need_dX=False)
+    assert torch.equal(dA4, r1[1]) and torch.equal(dB4, r1[2])
+
+
+def test_zero_adapter_reduces_to_dequant_matmul():
+    """B = 0: Y must equal X dequant(W)^T computed by the oracle, adapter grads still flow."""
+    inp = synth.layer_inputs("tiny", M=40, shape=(256, 512), r=8, seed=5)
+    inp["B"] = np.zeros_like(inp["B"])
+    res, errs = run_case(inp)
+    assert float(res["dA"].abs().max()) == 0.0
