@@ -250,7 +250,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int s = t % NSTAGE;
       const uint32_t ph = (t / NSTAGE) & 1;
       ok = mbar_wait(&full_tma[s], ph, abort_flag);
-      if (ok && kDeq && t >= n_lora) ok = mbar_wait(&full_w[s], ph, abort_flag);
+      // full_w[s] completes one phase per use of stage s (the dequant warps
+      // also arrive, without work, on adapter steps), so its parity is ph too
+      if (ok && kDeq) ok = mbar_wait(&full_w[s], ph, abort_flag);
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
@@ -301,9 +303,16 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
       };
       float c1_next = (n_main > 0) ? load_scale(step_begin) : 0.f;
-      for (int t = n_lora; t < total; ++t) {
+      for (int t = 0; t < total; ++t) {
         const int s = t % NSTAGE;
         const uint32_t ph = (t / NSTAGE) & 1;
+        if (t < n_lora) {
+          // adapter slice: B comes from TMA; keep full_w[s]'s phase count in
+          // step with the stage's uses (t < n_lora <= NSTAGE: first use)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_w[s]);
+          continue;
+        }
         const int ks = step_begin + (t - n_lora);
         const float c1 = c1_next;
         if (t + 1 < total) c1_next = load_scale(ks + 1);

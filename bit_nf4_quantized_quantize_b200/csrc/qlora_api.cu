@@ -186,6 +186,8 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
                 const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
   using L = GemmSmem<BN, NSTAGE, BSRC, NDW>;
   auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW>;
+  // the adapter slices must fit in the first pass over the stages
+  if (args.n_lora > NSTAGE) return QLORA_ERR_UNSUPPORTED_SHAPE;
   static bool attr_set[kMaxDevices];
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
