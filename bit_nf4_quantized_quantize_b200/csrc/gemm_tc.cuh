@@ -44,7 +44,7 @@ enum OutMode : int { kOutBf16 = 0, kOutF32Partial = 1 };
 
 constexpr int kBK = 64;                 // reduction elements per stage (128 B of bf16)
 constexpr int kBM = 128;                // MMA M
-constexpr int kATileBytes = kBM * kBK * 2;
+constexpr int kAHalfBytes = kBM * kBK * 2;  // one 128-row A half (16 KiB)
 
 struct GemmArgs {
   int m_rows;             // rows of D (MMA M side) in total
@@ -64,13 +64,16 @@ struct GemmArgs {
   int64_t split_stride;   // elements between splits (partial mode)
 };
 
-template <int BN, int NSTAGE, int BSRC, int NDW>
+template <int BN, int NSTAGE, int BSRC, int NDW, int MH>
 struct GemmSmem {
   static constexpr bool kDeq = (BSRC == kBDeqK || BSRC == kBDeqMN);
+  static constexpr int kATileBytes = MH * kAHalfBytes;
   static constexpr int kBTileBytes = BN * kBK * 2;
   static constexpr int kPTileBytes = kDeq ? BN * kBK / 2 : 0;
   static constexpr int kAOff = 0;
   static constexpr int kBOff = kAOff + NSTAGE * kATileBytes;
+  static_assert(kBOff + NSTAGE * (kBTileBytes + kPTileBytes) + 1024 + 8 * (3 * NSTAGE + 1) + 16 <= 232448,
+                "shared memory");
   static constexpr int kPOff = kBOff + NSTAGE * kBTileBytes;
   static constexpr int kBarOff = kPOff + NSTAGE * kPTileBytes;
   static constexpr int kNumBars = 3 * NSTAGE + 1;
@@ -144,19 +147,25 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 // ---------------------------------------------------------------------------
-template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW>
+// MH = number of 128-row halves of the M tile.  With MH = 2 the tile is
+// 256 x BN: two accumulators (TMEM columns [0, BN) and [BN, 2 BN)) share each
+// B tile, which halves the dequant work per MMA.
+template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW, int MH>
 __global__ void __launch_bounds__(64 + 32 * NDW, 1)
 qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                   const GemmArgs args) {
-  using L = GemmSmem<BN, NSTAGE, BSRC, NDW>;
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH>;
   constexpr bool kDeq = L::kDeq;
+  constexpr int kATileBytes = L::kATileBytes;
+  static_assert(MH == 1 || MH == 2, "MH");
+  static_assert(MH == 1 || !A_MN, "MN-major A uses one half");
   constexpr bool kBMN = (BSRC == kBTmaMN || BSRC == kBDeqMN);
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(!kDeq || NDW * 32 == BN, "one dequant item per thread");
   static_assert(NDW % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
   constexpr uint32_t kIdesc = idesc_bf16_m128(BN, A_MN ? 1u : 0u, kBMN ? 1u : 0u);
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kTmemCols = (MH * BN) < 32 ? 32 : MH * BN;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,7 +178,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
+  const int m0 = blockIdx.x * (kBM * MH);
   const int c0 = blockIdx.y * BN;
   const int split = blockIdx.z;
   const int step_begin = split * args.steps_per_split;
@@ -267,6 +276,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           const uint64_t bd = kBMN ? smem_desc_sw128(b_base + kk * 2048, kBK * 128)
                                    : smem_desc_sw128(b_base + kk * 32, 16);
           umma_bf16(tmem_d, ad, bd, kIdesc, (t > 0 || kk > 0) ? 1u : 0u);
+          if (MH == 2)
+            umma_bf16(tmem_d + BN, smem_desc_sw128(a_base + kAHalfBytes + kk * 32, 16), bd, kIdesc,
+                      (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
       }
@@ -302,7 +314,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int64_t blk = static_cast<int64_t>(wr) * args.w_kblocks + kb;
         return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
       };
-      float c1_next = (n_main > 0) ? load_scale(step_begin) : 0.f;
+      // scales are prefetched two steps ahead (c1_a: this step, c1_b: next)
+      float c1_a = (n_main > 0) ? load_scale(step_begin) : 0.f;
+      float c1_b = (n_main > 1) ? load_scale(step_begin + 1) : 0.f;
       for (int t = 0; t < total; ++t) {
         const int s = t % NSTAGE;
         const uint32_t ph = (t / NSTAGE) & 1;
@@ -314,8 +328,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           continue;
         }
         const int ks = step_begin + (t - n_lora);
-        const float c1 = c1_next;
-        if (t + 1 < total) c1_next = load_scale(ks + 1);
+        const float c1 = c1_a;
+        c1_a = c1_b;
+        if (t + 2 < total) c1_b = load_scale(ks + 2);
         const DeqTable tab = make_table(level, c1);
         if (!mbar_wait(&full_tma[s], ph, abort_flag)) { ok = false; break; }
         const uint32_t p_base = smem_u32(smem + L::kPOff + s * L::kPTileBytes);
@@ -355,36 +370,40 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       tc_fence_after();
       const int q = warp & 3;
       const int grp = (warp - 2) >> 2;
-      const int row = m0 + q * 32 + lane;
-      for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
-        tmem_ld_wait();
-        const int col = c0 + ch * 32;
-        if (row < args.m_rows && col < args.n_cols) {
-          if (OUT == kOutBf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
-                                                  static_cast<int64_t>(row) * args.ld_out + col);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 o;
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-              o.x = *reinterpret_cast<uint32_t*>(&h0);
-              o.y = *reinterpret_cast<uint32_t*>(&h1);
-              o.z = *reinterpret_cast<uint32_t*>(&h2);
-              o.w = *reinterpret_cast<uint32_t*>(&h3);
-              dst[i] = o;
-            }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
+#pragma unroll 1
+      for (int h = 0; h < MH; ++h) {
+        const int row = m0 + h * kBM + q * 32 + lane;
+#pragma unroll 1
+        for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + h * BN + ch * 32, v);
+          tmem_ld_wait();
+          const int col = c0 + ch * 32;
+          if (row < args.m_rows && col < args.n_cols) {
+            if (OUT == kOutBf16) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
                                                     static_cast<int64_t>(row) * args.ld_out + col);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+              for (int i = 0; i < 4; ++i) {
+                uint4 o;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                o.x = *reinterpret_cast<uint32_t*>(&h0);
+                o.y = *reinterpret_cast<uint32_t*>(&h1);
+                o.z = *reinterpret_cast<uint32_t*>(&h2);
+                o.w = *reinterpret_cast<uint32_t*>(&h3);
+                dst[i] = o;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
+                                                      static_cast<int64_t>(row) * args.ld_out + col);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
           }
         }
       }
@@ -392,14 +411,16 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       // a split with no work still owns its slice of the partial buffer: zero it
       const int q = warp & 3;
       const int grp = (warp - 2) >> 2;
-      const int row = m0 + q * 32 + lane;
-      for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
-        const int col = c0 + ch * 32;
-        if (row < args.m_rows && col < args.n_cols) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
-                                                  static_cast<int64_t>(row) * args.ld_out + col);
+      for (int h = 0; h < MH; ++h) {
+        const int row = m0 + h * kBM + q * 32 + lane;
+        for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
+          const int col = c0 + ch * 32;
+          if (row < args.m_rows && col < args.n_cols) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + split * args.split_stride +
+                                                    static_cast<int64_t>(row) * args.ld_out + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
       }
     }

@@ -181,11 +181,11 @@ int timed(int kind, cudaStream_t st, F&& launch) {
 }
 
 // ------------------------------------------------------------------ launches
-template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW>
+template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW, int MH = 1>
 int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                 const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
-  using L = GemmSmem<BN, NSTAGE, BSRC, NDW>;
-  auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW>;
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH>;
+  auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW, MH>;
   // the adapter slices must fit in the first pass over the stages
   if (args.n_lora > NSTAGE) return QLORA_ERR_UNSUPPORTED_SHAPE;
   static bool attr_set[kMaxDevices];
@@ -337,7 +337,7 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    quantize_dq_kernel<<<static_cast<unsigned>(groups), 256, 0, st>>>(W, n_blocks, codes, q8, s2, tables());
+    quantize_dq_kernel<<<static_cast<unsigned>(groups), kQuantThreads, 0, st>>>(W, n_blocks, codes, q8, s2, tables());
     return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
   });
 }
@@ -390,11 +390,15 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
 
   if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, part, L.pu, st, dev)) return rc;
 
+  // M tiles of 256 rows (two accumulators sharing each dequantized B tile)
+  // unless the whole batch fits in one 128-row tile
+  const bool two_halves = M > 128;
+  const uint32_t a_rows = two_halves ? 256 : 128;
   CUtensorMap tx, tp, tus, tb;
-  if (!map_bf16(&tx, X, M, k_in, 64, 128) ||
+  if (!map_bf16(&tx, X, M, k_in, 64, a_rows) ||
       !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 256,
                 CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 256))
+      !map_bf16(&tus, Us, M, r, 64, a_rows) || !map_bf16(&tb, B, n_out, r, 64, 256))
     return QLORA_ERR_CUDA;
   GemmArgs g{};
   g.m_rows = static_cast<int>(M);
@@ -410,8 +414,9 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   g.out = Y;
   g.ld_out = n_out;
   g.split_stride = 0;
-  const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256), 1);
-  return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8>(grid, tx, tp, tus, tb, g, st, dev);
+  const dim3 grid(static_cast<unsigned>((M + a_rows - 1) / a_rows), static_cast<unsigned>((n_out + 255) / 256), 1);
+  if (two_halves) return launch_gemm<256, 3, false, kBDeqK, kOutBf16, 8, 2>(grid, tx, tp, tus, tb, g, st, dev);
+  return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8, 1>(grid, tx, tp, tus, tb, g, st, dev);
 }
 
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
@@ -471,10 +476,12 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   }
   // dX = dY dequant(W) + (s V) A
   if (dX) {
+    const bool two_halves = M > 128;
+    const uint32_t a_rows = two_halves ? 256 : 128;
     CUtensorMap ta, tp, ta2, tb2;
-    if (!map_bf16(&ta, dY, M, N, 64, 128) ||
+    if (!map_bf16(&ta, dY, M, N, 64, a_rows) ||
         !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
+        !map_bf16(&ta2, Vs, M, r, 64, a_rows) || !map_bf16(&tb2, A, r, K, 64, 64))
       return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.m_rows = static_cast<int>(M);
@@ -489,8 +496,10 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     fill_levels(g);
     g.out = dX;
     g.ld_out = K;
-    const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256), 1);
-    if (int rc = launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8>(grid, ta, tp, ta2, tb2, g, st, dev)) return rc;
+    const dim3 grid(static_cast<unsigned>((M + a_rows - 1) / a_rows), static_cast<unsigned>((K + 255) / 256), 1);
+    const int rc = two_halves ? launch_gemm<256, 3, false, kBDeqMN, kOutBf16, 8, 2>(grid, ta, tp, ta2, tb2, g, st, dev)
+                              : launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
+    if (rc) return rc;
   }
   // dA^T = X^T V and dB = dY^T U, reduced over M in split partials
   float* part_a = part;

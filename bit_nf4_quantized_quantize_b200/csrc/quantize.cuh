@@ -4,12 +4,12 @@
 // NormalFloat levels, 4-bit code) and §5-2 (8-bit re-quantization of the fp32
 // absmax constants in groups of 256, one fp32 second-level constant).
 //
-// quantize_dq_kernel: one CTA per group of 256 blocks (16384 weights, 64 KiB
-// of fp32 input).  Eight threads share a 64-block (8 consecutive weights each,
-// two 16-byte loads), so a warp reads 1 KiB contiguous per pass; the block
-// absmax is a 3-step xor-shuffle max.  The nearest level comes from a
+// quantize_dq_kernel: one CTA of 512 threads per group of 256 blocks (16384
+// weights, 64 KiB of fp32 input).  Eight threads share a 64-block (8
+// consecutive weights each, two 16-byte loads), so a warp reads 1 KiB
+// contiguous per pass; the block absmax is a 3-step xor-shuffle max.  The nearest level comes from a
 // 257-cell lookup table over floor(128 * w_norm) (every cell of width 1/128
-// holds at most one decision threshold), so the search is one shared-memory
+// holds at most one decision threshold), so the search is one 8-byte shared-memory
 // load and one compare.  The group's 256 absmax values then stay in shared
 // memory for the second-level quantization, so the fp32 constants never go to
 // HBM.  Traffic per weight: 4 B read, 0.5 + 1/64 + 4/16384 B written.
@@ -30,32 +30,32 @@ struct Nf4Tables {
   uint8_t cell_lo[kLutCells];  // code of the cell's left edge
 };
 
-__global__ void __launch_bounds__(256)
+constexpr int kQuantThreads = 512;  // 16 warps; 8 threads per 64-block, 4 passes of 64 blocks
+
+__global__ void __launch_bounds__(kQuantThreads, 2)
 quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
                    uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
-  __shared__ float s_thr[kLutCells];
-  __shared__ int s_lo[kLutCells];
+  __shared__ int2 s_lut[kLutCells];   // {threshold bits, code of the cell's left edge}
   __shared__ float s_absmax[kGroup];
-  __shared__ float s_warpmax[8];
+  __shared__ float s_warpmax[kGroup / 32];
 
   const int tid = threadIdx.x;
-  for (int i = tid; i < kLutCells; i += blockDim.x) {
-    s_thr[i] = tabs.cell_thr[i];
-    s_lo[i] = tabs.cell_lo[i];
-  }
+  for (int i = tid; i < kLutCells; i += kQuantThreads)
+    s_lut[i] = make_int2(__float_as_int(tabs.cell_thr[i]), tabs.cell_lo[i]);
 
   const int64_t g = blockIdx.x;
   const int64_t b_first = g * kGroup;
   const int64_t left = n_blocks - b_first;
   const int nb = left < kGroup ? static_cast<int>(left) : kGroup;
   const int sub = tid & 7;     // 8 threads per 64-block
-  const int lb0 = tid >> 3;    // block within a pass (32 blocks per pass)
+  const int lb0 = tid >> 3;    // block within a pass (64 blocks per pass)
+  constexpr int kPasses = kGroup / (kQuantThreads / 8);
 
-  // Issue every load of the group up front (16 x 16 B per thread in flight).
-  float4 v[8][2];
+  // Issue every load of the thread up front (8 x 16 B in flight per thread).
+  float4 v[kPasses][2];
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int lb = p * 32 + lb0;
+  for (int p = 0; p < kPasses; ++p) {
+    const int lb = p * (kQuantThreads / 8) + lb0;
     if (lb < nb) {
       const float4* src = reinterpret_cast<const float4*>(W + (b_first + lb) * kBlock + sub * 8);
       v[p][0] = __ldcs(src);
@@ -68,10 +68,10 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
   __syncthreads();  // lookup table ready
 
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int lb = p * 32 + lb0;
-    float e[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
-                  v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
+  for (int p = 0; p < kPasses; ++p) {
+    const int lb = p * (kQuantThreads / 8) + lb0;
+    const float e[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
+                        v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
     float am = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(e[j]));
@@ -84,9 +84,11 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
       for (int j = 0; j < 8; ++j) {
         // one IEEE fp32 division, round to nearest (never the reciprocal form)
         const float wn = am > 0.f ? __fdiv_rn(e[j], am) : 0.f;
-        int cell = __float2int_rd(wn * 128.f) + 128;   // exact: scaling by 2^7
-        cell = min(max(cell, 0), kLutCells - 1);
-        const int code = s_lo[cell] + (wn >= s_thr[cell] ? 1 : 0);
+        // |wn| <= 1, so floor(128 wn) + 128 is in [0, 256]; the unsigned min
+        // only guards against NaN input (a caller error)
+        const unsigned cell = min(static_cast<unsigned>(__float2int_rd(wn * 128.f) + 128), 256u);
+        const int2 ent = s_lut[cell];
+        const int code = ent.y + (wn >= __int_as_float(ent.x) ? 1 : 0);
         packed |= static_cast<uint32_t>(code) << (4 * j);
       }
       *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
@@ -96,26 +98,31 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
   __syncthreads();
 
   // Second level: c2 = max of the group's absmax, s2 = fp32(c2/255),
-  // q = min(255, rint_half_even(fp32(absmax/s2))).
-  const float my = tid < nb ? s_absmax[tid] : 0.f;
-  float m = my;
+  // q = min(255, rint_half_even(fp32(absmax/s2))).  Threads 0..255 own one
+  // absmax each (warps 0..7).
+  if (tid < kGroup) {
+    const float my = tid < nb ? s_absmax[tid] : 0.f;
+    float m = my;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((tid & 31) == 0) s_warpmax[tid >> 5] = m;
-  __syncthreads();
-  float c2 = s_warpmax[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_warpmax[w]);
-  const float sc = __fdiv_rn(c2, 255.f);
-  if (tid < nb) {
-    int q = 0;
-    if (sc != 0.f) {
-      const float ratio = __fdiv_rn(my, sc);
-      q = min(255, __float2int_rn(ratio));  // round half to even
-    }
-    q8[b_first + tid] = static_cast<uint8_t>(q);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) s_warpmax[tid >> 5] = m;
   }
-  if (tid == 0) s2[g] = sc;
+  __syncthreads();
+  if (tid < kGroup) {
+    float c2 = s_warpmax[0];
+#pragma unroll
+    for (int w = 1; w < kGroup / 32; ++w) c2 = fmaxf(c2, s_warpmax[w]);
+    const float sc = __fdiv_rn(c2, 255.f);
+    if (tid < nb) {
+      int q = 0;
+      if (sc != 0.f) {
+        const float ratio = __fdiv_rn(s_absmax[tid], sc);
+        q = min(255, __float2int_rn(ratio));  // round half to even
+      }
+      q8[b_first + tid] = static_cast<uint8_t>(q);
+    }
+    if (tid == 0) s2[g] = sc;
+  }
 }
 
 // Dense dequantization: w = fp32(level[code] * fp32(q * s2)), fp32 or bf16 out.
