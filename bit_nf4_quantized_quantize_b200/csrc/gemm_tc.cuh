@@ -434,49 +434,4 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   }
 }
 
-// ---------------------------------------------------------------------------
-// Deterministic reductions of split partials (fixed split order).
-
-// U or V: P[split][M][rpad] -> plain (bf16, may be NULL) and scaled (bf16 of s*sum).
-__global__ void reduce_lora_kernel(const float* __restrict__ P, int splits, int64_t split_stride, int M,
-                                   int r, int rpad, float s, __nv_bfloat16* __restrict__ plain,
-                                   __nv_bfloat16* __restrict__ scaled) {
-  const int64_t n = static_cast<int64_t>(M) * r;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = i / r;
-    const int j = static_cast<int>(i - m * r);
-    float acc = 0.f;
-    for (int sp = 0; sp < splits; ++sp) acc += P[sp * split_stride + m * rpad + j];
-    if (plain) plain[i] = __float2bfloat16_rn(acc);
-    if (scaled) scaled[i] = __float2bfloat16_rn(s * acc);
-  }
-}
-
-// dA^T partials P[split][K][rpad] -> dA[r][K] = s * sum (transposed write);
-// dB partials Q[split][N][rpad] -> dB[N][r] = s * sum.
-__global__ void reduce_grad_kernel(const float* __restrict__ P, int splits_a, int64_t stride_a, int K,
-                                   const float* __restrict__ Q, int splits_b, int64_t stride_b, int N,
-                                   int r, int rpad, float s, float* __restrict__ dA, float* __restrict__ dB) {
-  const int64_t na = static_cast<int64_t>(r) * K;
-  const int64_t nb = static_cast<int64_t>(N) * r;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < na + nb;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    if (i < na) {
-      const int64_t j = i / K;
-      const int64_t k = i - j * K;
-      float acc = 0.f;
-      for (int sp = 0; sp < splits_a; ++sp) acc += P[sp * stride_a + k * rpad + j];
-      dA[i] = s * acc;
-    } else {
-      const int64_t e = i - na;
-      const int64_t n = e / r;
-      const int64_t j = e - n * r;
-      float acc = 0.f;
-      for (int sp = 0; sp < splits_b; ++sp) acc += Q[sp * stride_b + n * rpad + j];
-      dB[e] = s * acc;
-    }
-  }
-}
-
 }  // namespace qlora

@@ -1,0 +1,276 @@
+// Skinny adapter products of the QLoRA layer on tcgen05, split-K across a
+// thread-block cluster and reduced through distributed shared memory.
+//
+//   U    = X A^T      (M x r)   -> U (bf16) and s*U (bf16)      reduction over K
+//   V    = dY B       (M x r)   -> V (bf16) and s*V (bf16)      reduction over N
+//   dA^T = X^T V      (K x r)   -> dA = s * (.)^T  (fp32 r x K) reduction over M
+//   dB   = dY^T U     (N x r)   -> dB = s * (.)    (fp32 N x r) reduction over M
+//
+// ("逆伝播と勾配の流れ" of "QLoRAの理論と実装": dL/dB = (alpha/r) dL/dY (A X)^T and
+// dL/dA = (alpha/r) B^T dL/dY X^T, written row-major.)
+//
+// Each output tile is 128 rows x 64 columns (one 64-wide slice of r).  The S
+// CTAs of a cluster (S = 1, 2, 4 or 8, along grid z) take consecutive slices
+// of the reduction; after the mainloop each CTA copies its TMEM accumulator to
+// its own shared memory, the cluster synchronises, and CTA c sums rows
+// [c*128/S, (c+1)*128/S) over the S CTAs in rank order (deterministic) and
+// writes the final values.  No partial sums go to global memory and no
+// reduction kernel follows.  Two independent problems (dA and dB) can share
+// one launch: blockIdx.x below tiles0 selects problem 0.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "ptx_sm100.cuh"
+
+namespace qlora {
+
+constexpr int kLoraStages = 4;
+constexpr int kLoraBN = 64;
+constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+
+enum LoraOut : int {
+  kLoraOutPlainScaled = 0,  // bf16 out0 = sum (may be NULL), bf16 out1 = s * sum; row-major [rows][r]
+  kLoraOutTransposed = 1,   // fp32 out0[col][row] = s * sum  (dA from dA^T tiles)
+  kLoraOutRowMajor = 2,     // fp32 out0[row][col] = s * sum  (dB)
+};
+
+struct LoraProblem {
+  int rows;        // rows of D (M, K or N)
+  int k_steps;     // reduction steps of 64
+  int per_split;   // reduction steps per cluster rank
+  int tiles_m;     // 128-row tiles
+  int tiles_n;     // 64-column slices of r
+  int out_kind;
+  void* out0;
+  void* out1;
+  int ld_t;        // kLoraOutTransposed: elements between out0 rows (= rows)
+};
+
+struct LoraArgs {
+  LoraProblem p[2];
+  int tiles0;      // blocks of problem 0 along x (tiles_m * tiles_n)
+  int r;
+  float s;
+};
+
+struct LoraSmem {
+  static constexpr int kATile = 128 * 64 * 2;   // 16 KiB
+  static constexpr int kBTile = 64 * 64 * 2;    // 8 KiB
+  static constexpr int kAOff = 0;
+  static constexpr int kBOff = kAOff + kLoraStages * kATile;
+  static constexpr int kBarOff = kBOff + kLoraStages * kBTile;   // 96 KiB
+  static constexpr int kMiscOff = kBarOff + (2 * kLoraStages + 1) * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kDynBytes = kBytes + 1024;
+  static constexpr int kRedBytes = 128 * 64 * 4;  // fp32 accumulator copy (reuses the A stages)
+  static_assert(kRedBytes <= kBOff, "reduction buffer fits in the A stages");
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// A_MN: A operand MN-major (dA^T = X^T V, dB = dY^T U); else K-major (U, V).
+// B_MN: B operand MN-major (V = dY B and the gradient products); else K-major (U).
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kLoraThreads, 2)
+qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                  const LoraArgs args) {
+  using L = LoraSmem;
+  constexpr uint32_t kIdesc = idesc_bf16_m128(kLoraBN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
+  constexpr uint32_t kTxBytes = L::kATile + L::kBTile;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + kLoraStages;
+  uint64_t* accum_full = empty + kLoraStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int which = static_cast<int>(blockIdx.x) < args.tiles0 ? 0 : 1;
+  const LoraProblem P = which ? args.p[1] : args.p[0];
+  const CUtensorMap* tA = which ? &tmA1 : &tmA0;
+  const CUtensorMap* tB = which ? &tmB1 : &tmB0;
+  const int tile = static_cast<int>(blockIdx.x) - (which ? args.tiles0 : 0);
+  const int m0 = (tile / P.tiles_n) * 128;
+  const int c0 = (tile % P.tiles_n) * kLoraBN;
+  const int S = static_cast<int>(gridDim.z);     // cluster size along z
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int ks0 = rank * P.per_split;
+  const int n_steps = max(0, min(P.k_steps, ks0 + P.per_split) - ks0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLoraStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kLoraBN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  bool ok = true;
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(tA);
+      tma_prefetch_desc(tB);
+      for (int t = 0; t < n_steps; ++t) {
+        const int s = t % kLoraStages;
+        if (t >= kLoraStages && !mbar_wait(&empty[s], ((t / kLoraStages) - 1) & 1, abort_flag)) break;
+        const int ks = ks0 + t;
+        uint8_t* a_dst = smem + L::kAOff + s * L::kATile;
+        uint8_t* b_dst = smem + L::kBOff + s * L::kBTile;
+        mbar_arrive_expect_tx(&full[s], kTxBytes);
+        if (A_MN) {
+          tma_load_2d(a_dst, tA, &full[s], m0, ks * 64);
+          tma_load_2d(a_dst + 64 * 128, tA, &full[s], m0 + 64, ks * 64);
+        } else {
+          tma_load_2d(a_dst, tA, &full[s], ks * 64, m0);
+        }
+        if (B_MN) tma_load_2d(b_dst, tB, &full[s], c0, ks * 64);
+        else tma_load_2d(b_dst, tB, &full[s], ks * 64, c0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    for (int t = 0; t < n_steps; ++t) {
+      const int s = t % kLoraStages;
+      if (!mbar_wait(&full[s], (t / kLoraStages) & 1, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kATile);
+        const uint32_t b_base = smem_u32(smem + L::kBOff + s * L::kBTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 64 * 128) : smem_desc_sw128(a_base + kk * 32, 16);
+          const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 64 * 128) : smem_desc_sw128(b_base + kk * 32, 16);
+          umma_bf16(tmem_d, ad, bd, kIdesc, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) umma_commit(accum_full);
+    __syncwarp();
+  } else {
+    // copy the accumulator (or zeros, for a rank with no steps) to shared memory
+    ok = mbar_wait(accum_full, 0, abort_flag);
+    float* red = reinterpret_cast<float*>(smem + L::kAOff);
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < kLoraBN / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+        tmem_ld_wait();
+        // row-major [128][64] with the 16-byte chunk index rotated by the row
+        // to spread the stores over the banks
+        float4* dst = reinterpret_cast<float4*>(red + row * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c16 = ((ch * 8 + i) + row) & 15;
+          float4 val = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          if (n_steps == 0) val = make_float4(0.f, 0.f, 0.f, 0.f);
+          dst[c16] = val;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // every rank's accumulator is in its shared memory
+
+  if (warp >= 2 && !*abort_flag) {
+    // rows [rank*128/S, (rank+1)*128/S) of the tile, summed over ranks 0..S-1
+    const int t = threadIdx.x - 64;            // 0..127
+    const int rows_here = 128 / S;
+    const uint32_t red_base = smem_u32(smem + L::kAOff);
+    const int items = rows_here * 16;          // 16 four-column chunks per row
+    for (int it = t; it < items; it += 128) {
+      int lr, c16;
+      if (P.out_kind == kLoraOutTransposed) {  // lanes along rows: coalesced transposed stores
+        lr = it % rows_here;
+        c16 = it / rows_here;
+      } else {
+        lr = it / 16;
+        c16 = it % 16;
+      }
+      const int trow = rank * rows_here + lr;
+      const uint32_t off = static_cast<uint32_t>(trow * 64 + ((c16 + trow) & 15) * 4) * 4u;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p = 0; p < S; ++p) {
+        const float4 v = ld_cluster_v4(map_to_rank(red_base + off, p));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const int grow = m0 + trow;
+      const int gcol = c0 + c16 * 4;
+      if (grow < P.rows && gcol < args.r) {
+        const float s = args.s;
+        if (P.out_kind == kLoraOutPlainScaled) {
+          const int64_t o = static_cast<int64_t>(grow) * args.r + gcol;
+          if (P.out0) {
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y), h1 = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&h0);
+            u.y = *reinterpret_cast<uint32_t*>(&h1);
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(P.out0) + o) = u;
+          }
+          if (P.out1) {
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(s * acc.x, s * acc.y);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(s * acc.z, s * acc.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&h0);
+            u.y = *reinterpret_cast<uint32_t*>(&h1);
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(P.out1) + o) = u;
+          }
+        } else if (P.out_kind == kLoraOutRowMajor) {
+          *reinterpret_cast<float4*>(static_cast<float*>(P.out0) + static_cast<int64_t>(grow) * args.r + gcol) =
+              make_float4(s * acc.x, s * acc.y, s * acc.z, s * acc.w);
+        } else {
+          float* o = static_cast<float*>(P.out0);
+          o[static_cast<int64_t>(gcol + 0) * P.ld_t + grow] = s * acc.x;
+          o[static_cast<int64_t>(gcol + 1) * P.ld_t + grow] = s * acc.y;
+          o[static_cast<int64_t>(gcol + 2) * P.ld_t + grow] = s * acc.z;
+          o[static_cast<int64_t>(gcol + 3) * P.ld_t + grow] = s * acc.w;
+        }
+      }
+    }
+  }
+
+  cluster_sync_all();   // no rank leaves while another still reads its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, kLoraBN);
+  }
+}
+
+}  // namespace qlora

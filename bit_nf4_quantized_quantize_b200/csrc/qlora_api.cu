@@ -18,6 +18,7 @@
 #include "ptx_sm100.cuh"
 #include "quantize.cuh"
 #include "gemm_tc.cuh"
+#include "lora_tc.cuh"
 
 using namespace qlora;
 
@@ -205,49 +206,80 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
   });
 }
 
-struct SplitPlan {
-  int tiles_m, tiles_n, k_steps, splits, per_split;
-};
-
-SplitPlan plan_split(int64_t rows, int64_t cols_pad, int64_t k_steps, int bn, int num_sms) {
-  SplitPlan p;
-  p.tiles_m = static_cast<int>((rows + kBM - 1) / kBM);
-  p.tiles_n = static_cast<int>(cols_pad / bn);
-  p.k_steps = static_cast<int>(k_steps);
-  const int tiles = p.tiles_m * p.tiles_n;
-  const int target = 2 * num_sms;
-  int splits = std::max(1, std::min<int>(p.k_steps, (target + tiles - 1) / tiles));
-  p.per_split = (p.k_steps + splits - 1) / splits;
-  p.splits = (p.k_steps + p.per_split - 1) / p.per_split;
-  return p;
-}
-
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t us, v, vs, u, part, total;
-  SplitPlan pu, pv, pa, pb;
+  size_t us, v, vs, u, total;
 };
 
+// bf16 scratch of M x r each: s*U (forward adapter operand), V and s*V
+// (backward), U (recomputed when the caller passes no saved U).
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+  (void)N; (void)K; (void)num_sms;
   WsLayout w;
-  const int64_t rpad = (r + 63) / 64 * 64;
-  w.pu = plan_split(M, rpad, K / 64, 64, num_sms);
-  w.pv = plan_split(M, rpad, N / 64, 64, num_sms);
-  w.pa = plan_split(K, rpad, (M + 63) / 64, 64, num_sms);
-  w.pb = plan_split(N, rpad, (M + 63) / 64, 64, num_sms);
   const size_t mr = a256(static_cast<size_t>(M) * r * 2);
-  const size_t part_u = static_cast<size_t>(w.pu.splits) * M * rpad;
-  const size_t part_v = static_cast<size_t>(w.pv.splits) * M * rpad;
-  const size_t part_ab = static_cast<size_t>(w.pa.splits) * K * rpad + a256(static_cast<size_t>(w.pb.splits) * N * rpad * 4) / 4;
-  const size_t part = std::max(part_u, std::max(part_v, part_ab)) * 4;
   w.us = 0;
   w.v = w.us + mr;
   w.vs = w.v + mr;
   w.u = w.vs + mr;
-  w.part = w.u + mr;
-  w.total = w.part + a256(part);
+  w.total = w.u + mr;
   return w;
+}
+
+// Cluster size for a split-K adapter product: the largest power of two <= 8
+// that keeps tiles x S within one wave of 2 CTAs per SM and gives every rank
+// at least one reduction step.
+int pick_cluster(int tiles, int k_steps, int num_sms) {
+  int S = 1;
+  while (S < 8 && tiles * S * 2 <= 2 * num_sms && S * 2 <= k_steps) S *= 2;
+  return S;
+}
+
+template <bool A_MN, bool B_MN>
+int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
+                const LoraArgs& args, int tiles_total, int S, cudaStream_t st, int dev, int kind) {
+  auto kern = qlora_lora_kernel<A_MN, B_MN>;
+  static bool attr_set[kMaxDevices];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LoraSmem::kDynBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  return timed(kind, st, [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_total), 1, static_cast<unsigned>(S));
+    cfg.blockDim = dim3(kLoraThreads, 1, 1);
+    cfg.dynamicSmemBytes = LoraSmem::kDynBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = static_cast<unsigned>(S);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a0, b0, a1, b1, args) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+  });
+}
+
+LoraProblem lora_problem(int rows, int k_steps, int S, int rpad, int kind, void* out0, void* out1, int ld_t) {
+  LoraProblem p{};
+  p.rows = rows;
+  p.k_steps = k_steps;
+  p.per_split = (k_steps + S - 1) / S;
+  p.tiles_m = (rows + 127) / 128;
+  p.tiles_n = rpad / 64;
+  p.out_kind = kind;
+  p.out0 = out0;
+  p.out1 = out1;
+  p.ld_t = ld_t;
+  return p;
 }
 
 int check_weight(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K) {
@@ -273,31 +305,20 @@ void fill_levels(GemmArgs& g) {
 
 // U = X A^T into `plain` (bf16, may be NULL) and `scaled` = bf16(s U) (may be NULL).
 int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat, int r, float s,
-                  uint16_t* plain, uint16_t* scaled, float* part, const SplitPlan& p, cudaStream_t st,
-                  int dev) {
+                  uint16_t* plain, uint16_t* scaled, int num_sms, cudaStream_t st, int dev) {
   const int rpad = (r + 63) / 64 * 64;
   CUtensorMap ta, tb;
   if (!map_bf16(&ta, X, M, K, 64, 128) || !map_bf16(&tb, Amat, r, K, 64, 64)) return QLORA_ERR_CUDA;
-  GemmArgs g{};
-  g.m_rows = static_cast<int>(M);
-  g.n_cols = rpad;
-  g.k_steps = p.k_steps;
-  g.steps_per_split = p.per_split;
-  g.n_lora = 0;
-  g.out = part;
-  g.ld_out = rpad;
-  g.split_stride = M * rpad;
-  int rc = launch_gemm<64, 4, false, kBTmaK, kOutF32Partial, 4>(dim3(p.tiles_m, p.tiles_n, p.splits), ta, tb, ta,
-                                                                tb, g, st, dev);
-  if (rc) return rc;
-  const int64_t n = M * r;
-  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
-  return timed(QLORA_KERNEL_LORA_REDUCE, st, [&] {
-    reduce_lora_kernel<<<blocks, 256, 0, st>>>(part, p.splits, M * rpad, static_cast<int>(M), r, rpad, s,
-                                               reinterpret_cast<__nv_bfloat16*>(plain),
-                                               reinterpret_cast<__nv_bfloat16*>(scaled));
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-  });
+  const int k_steps = static_cast<int>(K / 64);
+  const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
+  const int S = pick_cluster(tiles, k_steps, num_sms);
+  LoraArgs la{};
+  la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, plain, scaled, 0);
+  la.p[1] = la.p[0];
+  la.tiles0 = tiles;
+  la.r = r;
+  la.s = s;
+  return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM);
 }
 
 }  // namespace
@@ -384,11 +405,10 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* Us = reinterpret_cast<uint16_t*>(ws + L.us);
-  float* part = reinterpret_cast<float*>(ws + L.part);
   const float s = alpha / static_cast<float>(r);
   const int rpad = (r + 63) / 64 * 64;
 
-  if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, part, L.pu, st, dev)) return rc;
+  if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, sms, st, dev)) return rc;
 
   // M tiles of 256 rows (two accumulators sharing each dequantized B tile)
   // unless the whole batch fits in one 128-row tile
@@ -439,7 +459,6 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   uint16_t* V = reinterpret_cast<uint16_t*>(ws + L.v);
   uint16_t* Vs = reinterpret_cast<uint16_t*>(ws + L.vs);
   uint16_t* Ubuf = reinterpret_cast<uint16_t*>(ws + L.u);
-  float* part = reinterpret_cast<float*>(ws + L.part);
   const float s = alpha / static_cast<float>(r);
   const int rpad = (r + 63) / 64 * 64;
   const int N = static_cast<int>(n_out), K = static_cast<int>(k_in);
@@ -448,30 +467,21 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   {
     CUtensorMap ta, tb;
     if (!map_bf16(&ta, dY, M, N, 64, 128) || !map_bf16(&tb, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.m_rows = static_cast<int>(M);
-    g.n_cols = rpad;
-    g.k_steps = L.pv.k_steps;
-    g.steps_per_split = L.pv.per_split;
-    g.out = part;
-    g.ld_out = rpad;
-    g.split_stride = M * rpad;
-    if (int rc = launch_gemm<64, 4, false, kBTmaMN, kOutF32Partial, 4>(dim3(L.pv.tiles_m, L.pv.tiles_n, L.pv.splits),
-                                                                      ta, tb, ta, tb, g, st, dev))
-      return rc;
-    const int64_t n = M * r;
-    if (int rc = timed(QLORA_KERNEL_LORA_REDUCE, st, [&] {
-          reduce_lora_kernel<<<static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)), 256, 0, st>>>(
-              part, L.pv.splits, M * rpad, static_cast<int>(M), r, rpad, s, reinterpret_cast<__nv_bfloat16*>(V),
-              reinterpret_cast<__nv_bfloat16*>(Vs));
-          return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-        }))
-      return rc;
+    const int k_steps = N / 64;
+    const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
+    const int S = pick_cluster(tiles, k_steps, sms);
+    LoraArgs la{};
+    la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, V, Vs, 0);
+    la.p[1] = la.p[0];
+    la.tiles0 = tiles;
+    la.r = r;
+    la.s = s;
+    if (int rc = launch_lora<false, true>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM)) return rc;
   }
   // U (from the forward, or recomputed)
   const uint16_t* U = U_saved;
   if (!U) {
-    if (int rc = run_lora_down(X, M, K, A, r, s, Ubuf, nullptr, part, L.pu, st, dev)) return rc;
+    if (int rc = run_lora_down(X, M, K, A, r, s, Ubuf, nullptr, sms, st, dev)) return rc;
     U = Ubuf;
   }
   // dX = dY dequant(W) + (s V) A
@@ -501,47 +511,24 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
                               : launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
     if (rc) return rc;
   }
-  // dA^T = X^T V and dB = dY^T U, reduced over M in split partials
-  float* part_a = part;
-  float* part_b = part + static_cast<size_t>(L.pa.splits) * K * rpad;
+  // dA^T = X^T V and dB = dY^T U in one grouped launch, reduced over M
   {
-    CUtensorMap ta, tb;
-    if (!map_bf16(&ta, X, M, K, 64, 64) || !map_bf16(&tb, V, M, r, 64, 64)) return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.m_rows = K;
-    g.n_cols = rpad;
-    g.k_steps = L.pa.k_steps;
-    g.steps_per_split = L.pa.per_split;
-    g.out = part_a;
-    g.ld_out = rpad;
-    g.split_stride = static_cast<int64_t>(K) * rpad;
-    if (int rc = launch_gemm<64, 4, true, kBTmaMN, kOutF32Partial, 4>(dim3(L.pa.tiles_m, L.pa.tiles_n, L.pa.splits),
-                                                                     ta, tb, ta, tb, g, st, dev))
-      return rc;
-  }
-  {
-    CUtensorMap ta, tb;
-    if (!map_bf16(&ta, dY, M, N, 64, 64) || !map_bf16(&tb, U, M, r, 64, 64)) return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.m_rows = N;
-    g.n_cols = rpad;
-    g.k_steps = L.pb.k_steps;
-    g.steps_per_split = L.pb.per_split;
-    g.out = part_b;
-    g.ld_out = rpad;
-    g.split_stride = static_cast<int64_t>(N) * rpad;
-    if (int rc = launch_gemm<64, 4, true, kBTmaMN, kOutF32Partial, 4>(dim3(L.pb.tiles_m, L.pb.tiles_n, L.pb.splits),
-                                                                     ta, tb, ta, tb, g, st, dev))
-      return rc;
-  }
-  {
-    const int64_t n = static_cast<int64_t>(r) * K + static_cast<int64_t>(N) * r;
-    if (int rc = timed(QLORA_KERNEL_GRAD_REDUCE, st, [&] {
-          reduce_grad_kernel<<<static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)), 256, 0, st>>>(
-              part_a, L.pa.splits, static_cast<int64_t>(K) * rpad, K, part_b, L.pb.splits,
-              static_cast<int64_t>(N) * rpad, N, r, rpad, s, dA, dB);
-          return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-        }))
+    CUtensorMap ta0, tb0, ta1, tb1;
+    if (!map_bf16(&ta0, X, M, K, 64, 64) || !map_bf16(&tb0, V, M, r, 64, 64) ||
+        !map_bf16(&ta1, dY, M, N, 64, 64) || !map_bf16(&tb1, U, M, r, 64, 64))
+      return QLORA_ERR_CUDA;
+    const int k_steps = static_cast<int>((M + 63) / 64);
+    const int tiles_a = ((K + 127) / 128) * (rpad / 64);
+    const int tiles_b = ((N + 127) / 128) * (rpad / 64);
+    const int S = pick_cluster(tiles_a + tiles_b, k_steps, sms);
+    LoraArgs la{};
+    la.p[0] = lora_problem(K, k_steps, S, rpad, kLoraOutTransposed, dA, nullptr, K);
+    la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0);
+    la.tiles0 = tiles_a;
+    la.r = r;
+    la.s = s;
+    if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, st, dev,
+                                         QLORA_KERNEL_GRAD_GEMM))
       return rc;
   }
   return QLORA_OK;
