@@ -19,6 +19,7 @@
 #include "quantize.cuh"
 #include "gemm_tc.cuh"
 #include "lora_tc.cuh"
+#include "fused2_tc.cuh"
 
 using namespace qlora;
 
@@ -203,6 +204,42 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
   return timed(kind, st, [&] {
     kern<<<grid, 64 + 32 * NDW, L::kDynBytes, st>>>(a, b, a2, b2, args);
     return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  });
+}
+
+// Fused dequant-GEMM on CTA pairs (cluster of 2), tile (256*MH) x 256.
+template <int BSRC, int MH>
+int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const CUtensorMap& a2,
+                const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
+  using L = PairSmem<MH>;
+  auto kern = qlora_fused_pair_kernel<BSRC, MH>;
+  static bool attr_set[kMaxDevices];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const int kind = (BSRC == kBDeqK) ? QLORA_KERNEL_FWD : QLORA_KERNEL_DX;
+  return timed(kind, st, [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * num_pairs), 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kDynBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a, p, a2, b2, args) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
   });
 }
 
@@ -410,16 +447,6 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
 
   if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, sms, st, dev)) return rc;
 
-  // M tiles of 256 rows (two accumulators sharing each dequantized B tile)
-  // unless the whole batch fits in one 128-row tile
-  const bool two_halves = M > 128;
-  const uint32_t a_rows = two_halves ? 256 : 128;
-  CUtensorMap tx, tp, tus, tb;
-  if (!map_bf16(&tx, X, M, k_in, 64, a_rows) ||
-      !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 256,
-                CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !map_bf16(&tus, Us, M, r, 64, a_rows) || !map_bf16(&tb, B, n_out, r, 64, 256))
-    return QLORA_ERR_CUDA;
   GemmArgs g{};
   g.m_rows = static_cast<int>(M);
   g.n_cols = static_cast<int>(n_out);
@@ -434,8 +461,26 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   g.out = Y;
   g.ld_out = n_out;
   g.split_stride = 0;
-  const dim3 grid(static_cast<unsigned>((M + a_rows - 1) / a_rows), static_cast<unsigned>((n_out + 255) / 256), 1);
-  if (two_halves) return launch_gemm<256, 3, false, kBDeqK, kOutBf16, 8, 2>(grid, tx, tp, tus, tb, g, st, dev);
+  if (M > 128) {
+    // CTA pairs: tile (256*MH) x 256, each CTA expanding 128 weight rows per step
+    const int mh = M > 256 ? 2 : 1;
+    CUtensorMap tx, tp, tus, tb;
+    if (!map_bf16(&tx, X, M, k_in, 64, 128) ||
+        !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 128))
+      return QLORA_ERR_CUDA;
+    const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * static_cast<int>((n_out + 255) / 256);
+    return mh == 2 ? launch_pair<kBDeqK, 2>(pairs, tx, tp, tus, tb, g, st, dev)
+                   : launch_pair<kBDeqK, 1>(pairs, tx, tp, tus, tb, g, st, dev);
+  }
+  CUtensorMap tx, tp, tus, tb;
+  if (!map_bf16(&tx, X, M, k_in, 64, 128) ||
+      !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 256,
+                CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 256))
+    return QLORA_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256), 1);
   return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8, 1>(grid, tx, tp, tus, tb, g, st, dev);
 }
 
@@ -486,13 +531,6 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   }
   // dX = dY dequant(W) + (s V) A
   if (dX) {
-    const bool two_halves = M > 128;
-    const uint32_t a_rows = two_halves ? 256 : 128;
-    CUtensorMap ta, tp, ta2, tb2;
-    if (!map_bf16(&ta, dY, M, N, 64, a_rows) ||
-        !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_bf16(&ta2, Vs, M, r, 64, a_rows) || !map_bf16(&tb2, A, r, K, 64, 64))
-      return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.m_rows = static_cast<int>(M);
     g.n_cols = K;
@@ -506,9 +544,26 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     fill_levels(g);
     g.out = dX;
     g.ld_out = K;
-    const dim3 grid(static_cast<unsigned>((M + a_rows - 1) / a_rows), static_cast<unsigned>((K + 255) / 256), 1);
-    const int rc = two_halves ? launch_gemm<256, 3, false, kBDeqMN, kOutBf16, 8, 2>(grid, ta, tp, ta2, tb2, g, st, dev)
-                              : launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
+    int rc;
+    if (M > 128) {
+      const int mh = M > 256 ? 2 : 1;
+      CUtensorMap ta, tp, ta2, tb2;
+      if (!map_bf16(&ta, dY, M, N, 64, 128) ||
+          !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+          !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
+        return QLORA_ERR_CUDA;
+      const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * ((K + 255) / 256);
+      rc = mh == 2 ? launch_pair<kBDeqMN, 2>(pairs, ta, tp, ta2, tb2, g, st, dev)
+                   : launch_pair<kBDeqMN, 1>(pairs, ta, tp, ta2, tb2, g, st, dev);
+    } else {
+      CUtensorMap ta, tp, ta2, tb2;
+      if (!map_bf16(&ta, dY, M, N, 64, 128) ||
+          !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
+        return QLORA_ERR_CUDA;
+      const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256), 1);
+      rc = launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
+    }
     if (rc) return rc;
   }
   // dA^T = X^T V and dB = dY^T U in one grouped launch, reduced over M
