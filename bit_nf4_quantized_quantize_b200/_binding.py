@@ -33,6 +33,10 @@ _SIGNATURES = {
                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_linear_bwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
@@ -192,6 +196,28 @@ def qlora_linear_fwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float
     _check(load().qlora_linear_fwd(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A), _ptr(B), r,
                                    float(alpha), _ptr(Y), _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)),
            "qlora_linear_fwd")
+    return Y
+
+
+def qlora_linear_fwd_noalloc(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float,
+                             Y=None, U_save=None, stream=None):
+    """qlora_linear_fwd using the library's fixed 4 MiB device scratch (no workspace, no allocation
+    inside the library; the binding still allocates Y here if the caller passes none)."""
+    nc, nb, ng = quant_sizes(n_out, k_in)
+    _dev(codes, torch.uint8, "codes", (nc,))
+    _dev(q8, torch.uint8, "q8", (nb,))
+    _dev(s2, torch.float32, "s2", (ng,))
+    M = X.shape[0]
+    r = A.shape[0]
+    _dev(X, torch.bfloat16, "X", (M, k_in))
+    _dev(A, torch.bfloat16, "A", (r, k_in))
+    _dev(B, torch.bfloat16, "B", (n_out, r))
+    Y = torch.empty(M, n_out, dtype=torch.bfloat16, device=X.device) if Y is None else _dev(Y, torch.bfloat16, "Y", (M, n_out))
+    if U_save is not None:
+        _dev(U_save, torch.bfloat16, "U_save", (M, r))
+    _check(load().qlora_linear_fwd_noalloc(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
+                                           _ptr(B), r, float(alpha), _ptr(Y), _ptr(U_save), _stream(stream)),
+           "qlora_linear_fwd_noalloc")
     return Y
 
 

@@ -358,6 +358,36 @@ int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat,
   return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM);
 }
 
+// ------------------------------------------------------------------ fixed scratch
+// Scratch of qlora_linear_fwd_noalloc: a file-scope device array, so that the
+// library never allocates for that entry point.  Every GPU that loads the
+// library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name only stands in for the symbol, so the address is looked up once
+// per device (with that device current) and cached.
+void* noalloc_scratch(int dev) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices];
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 // ======================================================================= ABI
@@ -482,6 +512,24 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     return QLORA_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256), 1);
   return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8, 1>(grid, tx, tp, tus, tb, g, st, dev);
+}
+
+// Forward with the library's own fixed scratch instead of a caller workspace:
+// for callers that cannot allocate device memory (see include/qlora_nf4.h).
+int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out,
+                             int64_t k_in, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B,
+                             int r, float alpha, uint16_t* Y, uint16_t* U_save, void* stream) {
+  if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
+  if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
+  if (!Y) return QLORA_ERR_INVALID_ARG;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const size_t need = ws_layout(M, n_out, k_in, r, sms).total;
+  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;  // beyond the fixed 4 MiB
+  void* scratch = noalloc_scratch(dev);
+  if (!scratch) return QLORA_ERR_CUDA;
+  return qlora_linear_fwd(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, Y, U_save, scratch,
+                          kNoAllocScratchBytes, stream);
 }
 
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,

@@ -128,6 +128,35 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward without any allocation (the pages have no counterpart; this is an
+ * integration aid).  Same computation, arguments and results as
+ * qlora_linear_fwd, but the scratch comes from a fixed device array inside the
+ * library instead of a caller workspace.  It is for callers that cannot call
+ * cudaMalloc or hand over a workspace: a host whose device memory is entirely
+ * owned by another allocator, or a latency-bound caller that cannot afford
+ * cudaMalloc's implicit device synchronisation.
+ *
+ * - Limit: the fixed scratch is 4 MiB per device, held by every GPU that loads
+ *   the library until the process exits.  A call with
+ *   qlora_workspace_bytes(M, N, K, r) > 4 MiB (M * r above about 524,288)
+ *   returns QLORA_ERR_WORKSPACE and enqueues nothing.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine,
+ *   as long as launch timing (qlora_timing_enable) is off, which is the default.
+ * - Set-up: the first call on a device looks up the scratch's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it.  Make that
+ *   first call before any stream capture.
+ * - Sharing: every call uses the same scratch, which keeps the last call's
+ *   contents.  Every element this path reads is written by the same call first,
+ *   so nothing needs clearing.  Calls that overlap on the GPU (different
+ *   streams, or different host threads) race on the scratch: serialise them.
+ */
+int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                             int64_t n_out, int64_t k_in,
+                             const uint16_t* X, int64_t M,
+                             const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             uint16_t* Y, uint16_t* U_save, void* stream);
+
+/*
  * Backward, "逆伝播と勾配の流れ" (W frozen, gradients reach A and B only):
  *
  *   V  = dY B                                  (M x r)
