@@ -55,12 +55,16 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
       ::"r"(smem_u32(bar)), "h"(cta_mask) : "memory");
 }
-// Release-arrive (cluster scope) on the mbarrier at the same offset in CTA `rank`.
+// Arrive on the mbarrier at the same offset in CTA `rank` of the cluster.
+// Default (release, CTA-scope) semantics: the operand tile it announces was
+// written to this CTA's shared memory and published to the async proxy by
+// fence.proxy.async beforehand, which is what the pair's MMA reads through.
+// (A release at cluster scope added ~0.6 us per k-step on this path.)
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}"
       ::"r"(smem_u32(bar)), "r"(rank) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
