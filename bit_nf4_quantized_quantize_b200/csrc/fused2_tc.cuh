@@ -135,7 +135,7 @@ template <int BSRC, int MH>
 __global__ void __launch_bounds__(kPairThreads, 1)
 qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
                         const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                        const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
   static_assert(BSRC == kBDeqK || BSRC == kBDeqMN, "dequant sources only");
   using L = PairSmem<MH>;
   constexpr int NST = L::kStages;
@@ -314,34 +314,51 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     if (ok) {
       tc_fence_after();
       const int q = warp & 3;
+      // This warp owns TMEM lanes 32q..32q+31 (its 32 output rows) and the
+      // 32-column chunks ch = wg, wg+2, wg+4, wg+6 of each half.  Each 32 x 32
+      // block is converted to bf16 into a private 2 KiB staging tile in the
+      // (now idle) stage memory and written by one TMA bulk tensor store,
+      // which also clips rows >= M and columns >= N.
+      uint8_t* stage = smem + (warp - 2) * (MH * 4 * 2048);
 #pragma unroll 1
       for (int h = 0; h < MH; ++h) {
-        const int row = m0 + 256 * h + 128 * static_cast<int>(rank) + q * 32 + lane;
-#pragma unroll 1
-        for (int ch = wg; ch < kPairN / 32; ch += 2) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + h * kPairN + ch * 32, v);
-          tmem_ld_wait();
-          const int col = c0 + ch * 32;
-          if (row < args.m_rows && col < args.n_cols) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
-                                                  static_cast<int64_t>(row) * args.ld_out + col);
+        uint32_t v[4][32];
+        const uint32_t tbase = tmem_d + (static_cast<uint32_t>(q * 32) << 16) + h * kPairN;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 o;
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-              o.x = *reinterpret_cast<uint32_t*>(&h0);
-              o.y = *reinterpret_cast<uint32_t*>(&h1);
-              o.z = *reinterpret_cast<uint32_t*>(&h2);
-              o.w = *reinterpret_cast<uint32_t*>(&h3);
-              dst[i] = o;
-            }
+        for (int j = 0; j < 4; ++j) tmem_ld_32x32b_x32(tbase + (wg + 2 * j) * 32, v[j]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // row `lane` of the block: 64 bytes, 16-byte chunk c at (c ^ ((lane >> 1) & 3))
+          const uint32_t blk = smem_u32(stage + (h * 4 + j) * 2048);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 o;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 0]), __uint_as_float(v[j][8 * i + 1]));
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 2]), __uint_as_float(v[j][8 * i + 3]));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 4]), __uint_as_float(v[j][8 * i + 5]));
+            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 6]), __uint_as_float(v[j][8 * i + 7]));
+            o.x = *reinterpret_cast<uint32_t*>(&h0);
+            o.y = *reinterpret_cast<uint32_t*>(&h1);
+            o.z = *reinterpret_cast<uint32_t*>(&h2);
+            o.w = *reinterpret_cast<uint32_t*>(&h3);
+            st_shared_v4(blk + lane * 64 + ((static_cast<uint32_t>(i) ^ ((lane >> 1) & 3)) << 4), o);
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int row0 = m0 + 256 * h + 128 * static_cast<int>(rank) + q * 32;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tma_store_2d(&tmOut, stage + (h * 4 + j) * 2048, c0 + (wg + 2 * j) * 32, row0);
+        }
       }
+      if (lane == 0) {
+        tma_store_commit();
+        tma_store_wait_read();
+      }
+      __syncwarp();
     }
   }
 

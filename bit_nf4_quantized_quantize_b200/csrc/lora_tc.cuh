@@ -185,19 +185,20 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
     const int row = q * 32 + lane;
     if (ok) {
       tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < kLoraBN / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
-        tmem_ld_wait();
-        // row-major [128][64] with the 16-byte chunk index rotated by the row
-        // to spread the stores over the banks
-        float4* dst = reinterpret_cast<float4*>(red + row * 64);
+      uint32_t v[2][32];   // both 32-column chunks in flight before one wait
+      tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16), v[0]);
+      tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + 32, v[1]);
+      tmem_ld_wait();
+      // row-major [128][64] with the 16-byte chunk index rotated by the row
+      // to spread the stores over the banks
+      float4* dst = reinterpret_cast<float4*>(red + row * 64);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int c16 = ((ch * 8 + i) + row) & 15;
-          float4 val = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          float4 val = make_float4(__uint_as_float(v[ch][4 * i]), __uint_as_float(v[ch][4 * i + 1]),
+                                   __uint_as_float(v[ch][4 * i + 2]), __uint_as_float(v[ch][4 * i + 3]));
           if (n_steps == 0) val = make_float4(0.f, 0.f, 0.f, 0.f);
           dst[c16] = val;
         }

@@ -211,6 +211,12 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
 template <int BSRC, int MH>
 int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const CUtensorMap& a2,
                 const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
+  // output: bf16 [m_rows x n_cols] (row stride ld_out), stored in 32 x 32 blocks with 64-byte swizzle
+  CUtensorMap out;
+  if (!make_map(&out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, args.out, static_cast<uint64_t>(args.n_cols),
+                static_cast<uint64_t>(args.m_rows), static_cast<uint64_t>(args.ld_out) * 2, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return QLORA_ERR_CUDA;
   using L = PairSmem<MH>;
   auto kern = qlora_fused_pair_kernel<BSRC, MH>;
   static bool attr_set[kMaxDevices];
@@ -235,7 +241,7 @@ int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a, p, a2, b2, args) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, a, p, a2, b2, out, args) != cudaSuccess) {
       cudaGetLastError();
       return QLORA_ERR_CUDA;
     }
