@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     lib_path,
     load,
     qlora_dequant,
+    qlora_launch_count,
     qlora_device_status,
     qlora_linear_bwd,
     qlora_linear_fwd,

@@ -45,6 +45,7 @@ _SIGNATURES = {
     "qlora_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_timing_enable": (ctypes.c_int, [ctypes.c_int]),
     "qlora_timing_collect": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]),
+    "qlora_launch_count": (ctypes.c_int64, []),
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "lora_gemm", "lora_reduce", "fwd_fused", "dx_fused", "grad_gemm",
@@ -268,3 +269,8 @@ def qlora_timing_collect() -> dict:
     _check(load().qlora_timing_collect(ms.ctypes.data_as(ctypes.c_void_p), cnt.ctypes.data_as(ctypes.c_void_p),
                                        len(KERNEL_KINDS)), "qlora_timing_collect")
     return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS) if cnt[i]}
+
+
+def qlora_launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(load().qlora_launch_count())

@@ -180,6 +180,7 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   cluster_barrier();     // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  griddep_wait();   // no global access before the previous grid is complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (each CTA its own halves)
@@ -311,6 +312,7 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
     // ------------------------------------------------------------ epilogue (own 128 rows per half)
     if (ok) ok = mbar_wait_cluster(accum_full, 0, abort_flag);
+    griddep_launch_dependents();
     if (ok) {
       tc_fence_after();
       const int q = warp & 3;

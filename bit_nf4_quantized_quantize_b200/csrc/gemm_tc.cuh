@@ -202,6 +202,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  griddep_wait();   // no global access before the previous grid is complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -366,6 +367,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait(accum_full, 0, abort_flag);
+    griddep_launch_dependents();
     if (ok && total > 0) {
       tc_fence_after();
       const int q = warp & 3;

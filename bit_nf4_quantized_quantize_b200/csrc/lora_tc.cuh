@@ -80,10 +80,13 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
   return d;
 }
+// Plain remote load (no memory clobber, so consecutive loads can be in
+// flight together); ordering against the peers' writes comes from the
+// cluster barrier that precedes every use.
 __device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
   return v;
 }
 
@@ -133,6 +136,7 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  griddep_wait();   // no global access before the previous grid is complete
 
   bool ok = true;
   if (warp == 0) {
@@ -180,6 +184,7 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   } else {
     // copy the accumulator (or zeros, for a rank with no steps) to shared memory
     ok = mbar_wait(accum_full, 0, abort_flag);
+    griddep_launch_dependents();
     float* red = reinterpret_cast<float*>(smem + L::kAOff);
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -227,11 +232,15 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
       }
       const int trow = rank * rows_here + lr;
       const uint32_t off = static_cast<uint32_t>(trow * 64 + ((c16 + trow) & 15) * 4) * 4u;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int p = 0; p < S; ++p) {
-        const float4 v = ld_cluster_v4(map_to_rank(red_base + off, p));
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
+      // issue all remote loads before the first add, then sum in rank order
+      float4 v[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        if (p < S) v[p] = ld_cluster_v4(map_to_rank(red_base + off, p));
+      float4 acc = v[0];
+#pragma unroll
+      for (int p = 1; p < 8; ++p)
+        if (p < S) { acc.x += v[p].x; acc.y += v[p].y; acc.z += v[p].z; acc.w += v[p].w; }
       const int grow = m0 + trow;
       const int gcol = c0 + c16 * 4;
       if (grow < P.rows && gcol < args.r) {

@@ -28,6 +28,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialisation: a grid may be
+// scheduled while the previous grid on the stream is still finishing.  Every
+// kernel executes griddep_wait() before its first global-memory access (read
+// or write), so only its prologue (barrier init, TMEM allocation, descriptor
+// prefetch) overlaps the previous grid; griddep_launch_dependents() lets the
+// next grid be scheduled once every CTA of this one has issued it or exited.
+// Both are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -12,7 +12,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "ptx_sm100.cuh"
@@ -170,8 +172,11 @@ cudaEvent_t take_event() {
 
 // Run `launch` (which enqueues one kernel on st); bracket it with events when
 // timing is on.
+std::atomic<int64_t> g_launch_count{0};
+
 template <class F>
 int timed(int kind, cudaStream_t st, F&& launch) {
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
   if (!g_timing_on) return launch();
   std::lock_guard<std::mutex> lk(g_timing_mu);
   cudaEvent_t a = take_event(), b = take_event();
@@ -183,6 +188,37 @@ int timed(int kind, cudaStream_t st, F&& launch) {
 }
 
 // ------------------------------------------------------------------ launches
+// Launch with programmatic stream serialisation (see griddep_wait in
+// ptx_sm100.cuh), optionally as clusters of cluster_x x 1 x cluster_z CTAs.
+template <typename... KArgs, typename... Args>
+int launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cluster_x,
+              unsigned cluster_z, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x * cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
 template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW, int MH = 1>
 int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                 const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
@@ -202,8 +238,7 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
                  : (BSRC == kBDeqMN) ? QLORA_KERNEL_DX
                  : A_MN ? QLORA_KERNEL_GRAD_GEMM : QLORA_KERNEL_LORA_GEMM;
   return timed(kind, st, [&] {
-    kern<<<grid, 64 + 32 * NDW, L::kDynBytes, st>>>(a, b, a2, b2, args);
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+    return launch_ex(kern, grid, dim3(64 + 32 * NDW), L::kDynBytes, st, 1, 1, a, b, a2, b2, args);
   });
 }
 
@@ -229,23 +264,8 @@ int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const
   }
   const int kind = (BSRC == kBDeqK) ? QLORA_KERNEL_FWD : QLORA_KERNEL_DX;
   return timed(kind, st, [&] {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * num_pairs), 1, 1);
-    cfg.blockDim = dim3(kPairThreads, 1, 1);
-    cfg.dynamicSmemBytes = L::kDynBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a, p, a2, b2, out, args) != cudaSuccess) {
-      cudaGetLastError();
-      return QLORA_ERR_CUDA;
-    }
-    return QLORA_OK;
+    return launch_ex(kern, dim3(static_cast<unsigned>(2 * num_pairs)), dim3(kPairThreads), L::kDynBytes, st, 2, 1,
+                     a, p, a2, b2, out, args);
   });
 }
 
@@ -291,23 +311,8 @@ int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap&
     attr_set[dev] = true;
   }
   return timed(kind, st, [&] {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles_total), 1, static_cast<unsigned>(S));
-    cfg.blockDim = dim3(kLoraThreads, 1, 1);
-    cfg.dynamicSmemBytes = LoraSmem::kDynBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = static_cast<unsigned>(S);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a0, b0, a1, b1, args) != cudaSuccess) {
-      cudaGetLastError();
-      return QLORA_ERR_CUDA;
-    }
-    return QLORA_OK;
+    return launch_ex(kern, dim3(static_cast<unsigned>(tiles_total), 1, static_cast<unsigned>(S)), dim3(kLoraThreads),
+                     LoraSmem::kDynBytes, st, 1, static_cast<unsigned>(S), a0, b0, a1, b1, args);
   });
 }
 
@@ -431,8 +436,8 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    quantize_dq_kernel<<<static_cast<unsigned>(groups), kQuantThreads, 0, st>>>(W, n_blocks, codes, q8, s2, tables());
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+    return launch_ex(quantize_dq_kernel, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1, 1, W,
+                     n_blocks, codes, q8, s2, tables());
   });
 }
 
@@ -449,10 +454,10 @@ int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2, int6
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_DEQUANT, st, [&] {
     if (out_dtype == QLORA_OUT_BF16)
-      dequant_kernel<true><<<blocks, 256, 0, st>>>(codes, q8, s2, n_oct, out, tables());
-    else
-      dequant_kernel<false><<<blocks, 256, 0, st>>>(codes, q8, s2, n_oct, out, tables());
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+      return launch_ex(dequant_kernel<true>, dim3(blocks), dim3(256), 0, st, 1, 1, codes, q8, s2, n_oct, out,
+                       tables());
+    return launch_ex(dequant_kernel<false>, dim3(blocks), dim3(256), 0, st, 1, 1, codes, q8, s2, n_oct, out,
+                     tables());
   });
 }
 
@@ -642,6 +647,8 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   }
   return QLORA_OK;
 }
+
+int64_t qlora_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 
 int qlora_timing_enable(int on) {
   std::lock_guard<std::mutex> lk(g_timing_mu);

@@ -16,6 +16,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include "ptx_sm100.cuh"
 
 namespace qlora {
 
@@ -51,6 +52,7 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
   const int lb0 = tid >> 3;    // block within a pass (64 blocks per pass)
   constexpr int kPasses = kGroup / (kQuantThreads / 8);
 
+  griddep_wait();   // the previous grid's writes are visible from here on
   // Issue every load of the thread up front (8 x 16 B in flight per thread).
   float4 v[kPasses][2];
 #pragma unroll
@@ -95,6 +97,7 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
       if (sub == 0) s_absmax[lb] = am;
     }
   }
+  griddep_launch_dependents();
   __syncthreads();
 
   // Second level: c2 = max of the group's absmax, s2 = fp32(c2/255),
@@ -135,6 +138,7 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8
   __shared__ float s_level[16];
   if (threadIdx.x < 16) s_level[threadIdx.x] = tabs.level[threadIdx.x];
   __syncthreads();
+  griddep_wait();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_oct;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(codes) + i);

@@ -205,6 +205,9 @@ int qlora_device_status(void* stream);
 #define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
 #define QLORA_KERNEL_COUNT 8
 int qlora_timing_enable(int on);
+/* Number of kernels the library has enqueued since it was loaded (all
+ * devices, all streams), counted whether or not timing is enabled. */
+int64_t qlora_launch_count(void);
 int qlora_timing_collect(double* ms, int64_t* counts, int n_kinds);
 
 #ifdef __cplusplus
