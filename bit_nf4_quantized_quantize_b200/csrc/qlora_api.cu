@@ -71,16 +71,29 @@ Nf4Tables build_tables() {
     if (static_cast<double>(f) <= mid) f = std::nextafter(f, INFINITY);
     thr[i] = f;
   }
+  // cells of width 1/16: cell c covers [(c-16)/16, (c-15)/16)
+  T.fast_ok = 1;
   for (int c = 0; c < kLutCells; ++c) {
-    const double lo = (c - 128) / 128.0, hi = (c - 127) / 128.0;
-    int cnt = 0;
+    const double lo = (c - 16) / 16.0, hi = (c - 15) / 16.0;
+    int cnt = 0, inside_n = 0;
     float inside = INFINITY;
     for (int i = 0; i < 15; ++i) {
       if (thr[i] <= lo) ++cnt;
-      else if (thr[i] < hi) inside = std::min(inside, thr[i]);
+      else if (thr[i] < hi) { inside = std::min(inside, thr[i]); ++inside_n; }
     }
-    T.cell_lo[c] = static_cast<uint8_t>(cnt);
+    T.cell_lo[c] = cnt;
     T.cell_thr[c] = inside;
+    if (inside_n > 1) T.fast_ok = 0;  // (cannot happen for this table: thresholds are >= 0.088 apart)
+    // fast entry: threshold (4.0 when the cell has none) with the code in its 4 low bits
+    uint32_t bits;
+    const float f = std::isinf(inside) ? 4.0f : inside;
+    std::memcpy(&bits, &f, 4);
+    T.cell_fast[c] = (bits & ~15u) | static_cast<uint32_t>(cnt);
+  }
+  // every threshold must be farther than 2^-17 from every cell edge
+  for (int i = 0; i < 15; ++i) {
+    const double d = std::fabs(thr[i] * 16.0 - std::nearbyint(thr[i] * 16.0)) / 16.0;
+    if (d <= std::ldexp(1.0, -17)) T.fast_ok = 0;
   }
   return T;
 }

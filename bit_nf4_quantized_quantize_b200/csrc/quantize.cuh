@@ -7,12 +7,24 @@
 // quantize_dq_kernel: one CTA of 512 threads per group of 256 blocks (16384
 // weights, 64 KiB of fp32 input).  Eight threads share a 64-block (8
 // consecutive weights each, two 16-byte loads), so a warp reads 1 KiB
-// contiguous per pass; the block absmax is a 3-step xor-shuffle max.  The nearest level comes from a
-// 257-cell lookup table over floor(128 * w_norm) (every cell of width 1/128
-// holds at most one decision threshold), so the search is one 8-byte shared-memory
-// load and one compare.  The group's 256 absmax values then stay in shared
-// memory for the second-level quantization, so the fp32 constants never go to
-// HBM.  Traffic per weight: 4 B read, 0.5 + 1/64 + 4/16384 B written.
+// contiguous per pass; the block absmax is a 3-step xor-shuffle max.  The
+// group's 256 absmax values then stay in shared memory for the second-level
+// quantization, so the fp32 constants never go to HBM.  Traffic per weight:
+// 4 B read, 0.5 + 1/64 + 4/16384 B written.
+//
+// Nearest level.  The code of n = fp32(w / absmax) is #{i : n >= thr_i}, thr_i
+// the smallest fp32 above the exact midpoint of levels i and i+1.  Cells of
+// width 1/16 over [-1, 1] hold at most one threshold each (the thresholds are
+// >= 0.088 apart), so code = lo[cell] + (n >= thr[cell]) with cell =
+// floor(16 n) + 16.  Fast path: q0 = fp32(w * fp32(1/absmax)) is within 2.5
+// ulp of n, so every threshold that is not within 2^-18 of q0 lies on the
+// same side of q0 and n; the fast table packs the cell's left-edge code into
+// the 4 low mantissa bits of its threshold (a perturbation below 2^-19) and
+// one 4-byte shared-memory load serves the lookup.  When q0 is within 2^-18 of
+// the cell's threshold, or absmax is outside [2^-125, 2^125], the weight takes
+// the exact path: one IEEE division and the exact table.  The host checks
+// that no threshold lies within 2^-17 of a cell edge and otherwise disables
+// the fast path.  The result always equals the exact-division code.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -22,13 +34,16 @@ namespace qlora {
 
 constexpr int kBlock = 64;     // first-level block
 constexpr int kGroup = 256;    // second-level group (blocks per s2)
-constexpr int kLutCells = 257; // floor(128 n) + 128 for n in [-1, 1]
+constexpr int kLutCells = 33;  // floor(16 n) + 16 for n in [-1, 1]
+constexpr float kFastGuard = 3.814697265625e-06f;  // 2^-18
 
 // Host-built tables handed to the kernels by value.
 struct Nf4Tables {
   float level[16];             // NF4 levels, ascending (fp32)
-  float cell_thr[kLutCells];   // the decision threshold inside the cell, or +inf
-  uint8_t cell_lo[kLutCells];  // code of the cell's left edge
+  float cell_thr[kLutCells];   // exact threshold inside the cell, or +inf
+  int cell_lo[kLutCells];      // code of the cell's left edge
+  uint32_t cell_fast[kLutCells];  // threshold bits (or 4.0f) with the low 4 bits = cell_lo
+  int fast_ok;                 // the fast path's preconditions hold for this table
 };
 
 constexpr int kQuantThreads = 512;  // 16 warps; 8 threads per 64-block, 4 passes of 64 blocks
@@ -36,13 +51,17 @@ constexpr int kQuantThreads = 512;  // 16 warps; 8 threads per 64-block, 4 passe
 __global__ void __launch_bounds__(kQuantThreads, 2)
 quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
                    uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
-  __shared__ int2 s_lut[kLutCells];   // {threshold bits, code of the cell's left edge}
+  __shared__ int2 s_exact[kLutCells];     // {threshold bits, left-edge code}
+  __shared__ uint32_t s_fast[kLutCells];
   __shared__ float s_absmax[kGroup];
   __shared__ float s_warpmax[kGroup / 32];
 
   const int tid = threadIdx.x;
-  for (int i = tid; i < kLutCells; i += kQuantThreads)
-    s_lut[i] = make_int2(__float_as_int(tabs.cell_thr[i]), tabs.cell_lo[i]);
+  if (tid < kLutCells) {
+    s_exact[tid] = make_int2(__float_as_int(tabs.cell_thr[tid]), tabs.cell_lo[tid]);
+    s_fast[tid] = tabs.cell_fast[tid];
+  }
+  const bool fast_table = tabs.fast_ok != 0;
 
   const int64_t g = blockIdx.x;
   const int64_t b_first = g * kGroup;
@@ -81,16 +100,31 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
     if (lb < nb) {
+      // fast path needs fp32(1/absmax) to be a normal number
+      const bool fast = fast_table && am >= 2.35098870e-38f * 4.0f && am <= 4.2535296e37f;
+      const float rcp = fast ? __frcp_rn(am) : 0.f;
       uint32_t packed = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        // one IEEE fp32 division, round to nearest (never the reciprocal form)
-        const float wn = am > 0.f ? __fdiv_rn(e[j], am) : 0.f;
-        // |wn| <= 1, so floor(128 wn) + 128 is in [0, 256]; the unsigned min
-        // only guards against NaN input (a caller error)
-        const unsigned cell = min(static_cast<unsigned>(__float2int_rd(wn * 128.f) + 128), 256u);
-        const int2 ent = s_lut[cell];
-        const int code = ent.y + (wn >= __int_as_float(ent.x) ? 1 : 0);
+        int code;
+        bool exact = !fast;
+        if (fast) {
+          const float q0 = __fmul_rn(e[j], rcp);
+          const unsigned cell = min(static_cast<unsigned>(__float2int_rd(q0 * 16.f) + 16), 32u);
+          const uint32_t ent = s_fast[cell];
+          const float thr = __uint_as_float(ent);
+          code = static_cast<int>(ent & 15u) + (q0 >= thr ? 1 : 0);
+          exact = fabsf(q0 - thr) <= kFastGuard;
+        }
+        if (exact) {
+          // one IEEE fp32 division, round to nearest (never the reciprocal form)
+          const float wn = am > 0.f ? __fdiv_rn(e[j], am) : 0.f;
+          // |wn| <= 1, so floor(16 wn) + 16 is in [0, 32]; the unsigned min
+          // only guards against NaN input (a caller error)
+          const unsigned cell = min(static_cast<unsigned>(__float2int_rd(wn * 16.f) + 16), 32u);
+          const int2 ent = s_exact[cell];
+          code = ent.y + (wn >= __int_as_float(ent.x) ? 1 : 0);
+        }
         packed |= static_cast<uint32_t>(code) << (4 * j);
       }
       *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
