@@ -186,6 +186,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int n_main = max(0, step_end - step_begin);
   const int n_lora = (split == 0) ? args.n_lora : 0;
   const int total = n_lora + n_main;
+  // bf16 output with the reduction split over a cluster along z (the launch
+  // sets cluster dims (1, 1, gridDim.z)); MH == 1 only
+  const bool csplit = (OUT == kOutBf16) && MH == 1 && gridDim.z > 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -322,8 +325,11 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int s = t % NSTAGE;
         const uint32_t ph = (t / NSTAGE) & 1;
         if (t < n_lora) {
-          // adapter slice: B comes from TMA; keep full_w[s]'s phase count in
-          // step with the stage's uses (t < n_lora <= NSTAGE: first use)
+          // adapter slice: B comes from TMA.  Wait for the stage's bytes like
+          // any step (so these warps never run a phase ahead: a wait on a
+          // later phase of a barrier whose current phase is incomplete would
+          // return at once), then keep full_w[s]'s phase count in step.
+          if (!mbar_wait(&full_tma[s], ph, abort_flag)) { ok = false; break; }
           __syncwarp();
           if (lane == 0) mbar_arrive(&full_w[s]);
           continue;
@@ -368,7 +374,34 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait(accum_full, 0, abort_flag);
     griddep_launch_dependents();
-    if (ok && total > 0) {
+    if (ok && csplit) {
+      // split-K over the cluster: copy the tile's valid rows to this CTA's
+      // shared memory (fp32 [128][BN], 16-byte chunks rotated by the row);
+      // they are summed across the cluster below
+      float* red = reinterpret_cast<float*>(smem);
+      const int q = warp & 3;
+      const int grp = (warp - 2) >> 2;
+      const int m_valid = min(kBM, args.m_rows - m0);
+      if (q * 32 < m_valid) {
+        tc_fence_after();
+        const int row = q * 32 + lane;
+        for (int ch = grp; ch < BN / 32; ch += NDW / 4) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+          tmem_ld_wait();
+          if (row < m_valid) {
+            float4* dst = reinterpret_cast<float4*>(red + row * BN);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 val = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+              if (total == 0) val = make_float4(0.f, 0.f, 0.f, 0.f);
+              dst[(ch * 8 + i + row) & (BN / 4 - 1)] = val;
+            }
+          }
+        }
+      }
+    } else if (ok && total > 0) {
       tc_fence_after();
       const int q = warp & 3;
       const int grp = (warp - 2) >> 2;
@@ -430,6 +463,42 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
+  if (csplit) {
+    cluster_sync_all();   // every rank's partial tile is in its shared memory
+    if (warp >= 2 && !*abort_flag) {
+      // rank r sums its share of the valid rows' float4s over all ranks, in rank order
+      const int S = static_cast<int>(gridDim.z);
+      const int rank = static_cast<int>(cluster_ctarank());
+      const int m_valid = min(kBM, args.m_rows - m0);
+      const int n4 = m_valid * (BN / 4);
+      const int lo = static_cast<int>((static_cast<int64_t>(n4) * rank) / S);
+      const int hi = static_cast<int>((static_cast<int64_t>(n4) * (rank + 1)) / S);
+      const uint32_t red_base = smem_u32(smem);
+      for (int idx = lo + static_cast<int>(threadIdx.x) - 64; idx < hi; idx += 32 * NDW) {
+        const int row = idx / (BN / 4);
+        const int c4 = idx - row * (BN / 4);
+        const uint32_t off = static_cast<uint32_t>(row * BN + ((c4 + row) & (BN / 4 - 1)) * 4) * 4u;
+        float4 v[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p < S) v[p] = ld_cluster_v4(map_to_rank(red_base + off, p));
+        float4 a = v[0];
+#pragma unroll
+        for (int p = 1; p < 8; ++p)
+          if (p < S) { a.x += v[p].x; a.y += v[p].y; a.z += v[p].z; a.w += v[p].w; }
+        const int col = c0 + 4 * c4;
+        if (col < args.n_cols) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y), h1 = __floats2bfloat162_rn(a.z, a.w);
+          uint2 u;
+          u.x = *reinterpret_cast<uint32_t*>(&h0);
+          u.y = *reinterpret_cast<uint32_t*>(&h1);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(args.out) +
+                                    static_cast<int64_t>(m0 + row) * args.ld_out + col) = u;
+        }
+      }
+    }
+    cluster_sync_all();   // no rank leaves while another still reads its shared memory
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_d, kTmemCols);

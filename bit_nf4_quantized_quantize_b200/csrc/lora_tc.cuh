@@ -67,29 +67,6 @@ struct LoraSmem {
   static_assert(kRedBytes <= kBOff, "reduction buffer fits in the A stages");
 };
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t d;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
-  return d;
-}
-// Plain remote load (no memory clobber, so consecutive loads can be in
-// flight together); ordering against the peers' writes comes from the
-// cluster barrier that precedes every use.
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
-
 // A_MN: A operand MN-major (dA^T = X^T V, dB = dY^T U); else K-major (U, V).
 // B_MN: B operand MN-major (V = dY B and the gradient products); else K-major (U).
 template <bool A_MN, bool B_MN>

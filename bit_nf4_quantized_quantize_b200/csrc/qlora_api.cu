@@ -251,7 +251,7 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
                  : (BSRC == kBDeqMN) ? QLORA_KERNEL_DX
                  : A_MN ? QLORA_KERNEL_GRAD_GEMM : QLORA_KERNEL_LORA_GEMM;
   return timed(kind, st, [&] {
-    return launch_ex(kern, grid, dim3(64 + 32 * NDW), L::kDynBytes, st, 1, 1, a, b, a2, b2, args);
+    return launch_ex(kern, grid, dim3(64 + 32 * NDW), L::kDynBytes, st, 1, grid.z, a, b, a2, b2, args);
   });
 }
 
@@ -300,6 +300,15 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms) {
   w.u = w.vs + mr;
   w.total = w.u + mr;
   return w;
+}
+
+// Cluster size for the small-M split of the single-CTA fused kernel (one CTA
+// per SM): the most ranks (<= 8) that keep tiles x S within one wave and give
+// every rank at least two reduction steps.
+int pick_split(int tiles, int k_steps, int num_sms) {
+  int S = 1;
+  while (S < 8 && tiles * (S + 1) <= num_sms && (S + 1) * 2 <= k_steps) ++S;
+  return S;
 }
 
 // Cluster size for a split-K adapter product: the largest power of two <= 8
@@ -534,7 +543,12 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
                 CU_TENSOR_MAP_SWIZZLE_32B) ||
       !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 256))
     return QLORA_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256), 1);
+  // small M: split the reduction over a cluster of up to 8 CTAs (DSMEM sum)
+  const int tiles = static_cast<int>((M + 127) / 128) * static_cast<int>((n_out + 255) / 256);
+  const int S = pick_split(tiles, g.k_steps, sms);
+  g.steps_per_split = (g.k_steps + S - 1) / S;
+  const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256),
+                  static_cast<unsigned>(S));
   return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8, 1>(grid, tx, tp, tus, tb, g, st, dev);
 }
 
@@ -633,7 +647,11 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
           !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
         return QLORA_ERR_CUDA;
-      const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256), 1);
+      const int tiles = static_cast<int>((M + 127) / 128) * ((K + 255) / 256);
+      const int S = pick_split(tiles, g.k_steps, sms);
+      g.steps_per_split = (g.k_steps + S - 1) / S;
+      const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256),
+                      static_cast<unsigned>(S));
       rc = launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
     }
     if (rc) return rc;

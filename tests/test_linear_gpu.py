@@ -107,3 +107,13 @@ def test_zero_adapter_reduces_to_dequant_matmul():
     inp["B"] = np.zeros_like(inp["B"])
     res, errs = run_case(inp)
     assert float(res["dA"].abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 512, 256), (200, 512, 512)])
+def test_adapter_slices_filling_every_stage_back_to_back(M, N, K):
+    """r = 256 gives as many adapter slices as pipeline stages.  Two calls in a
+    row on the same shape with different weights: a stage read before its
+    bytes land would return the previous call's data, so the second call
+    checks the pipeline's phase handling, not just the arithmetic."""
+    for seed in (301, 302):
+        run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=256, seed=seed))
