@@ -49,7 +49,7 @@ _SIGNATURES = {
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "lora_gemm", "lora_reduce", "fwd_fused", "dx_fused", "grad_gemm",
-                "grad_reduce"]
+                "grad_reduce", "fwd_decode"]
 
 
 class QloraError(RuntimeError):

@@ -22,6 +22,7 @@
 #include "gemm_tc.cuh"
 #include "lora_tc.cuh"
 #include "fused2_tc.cuh"
+#include "decode_tc.cuh"
 
 using namespace qlora;
 
@@ -282,6 +283,91 @@ int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const
   });
 }
 
+// Small-M forward (decode_tc.cuh): row tiles of T = 128 - r weight rows, the
+// K range split over a cluster of S CTAs.  S is the largest cluster size
+// (<= 8) for which every row tile's cluster is resident at once (the
+// occupancy query accounts for how clusters pack into the GPU's processing
+// clusters) and every rank gets at least two k-steps.
+template <int MP>
+int launch_decode(const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& ta, const CUtensorMap& tb,
+                  DecodeArgs& d, cudaStream_t st, int dev) {
+  using L = DecodeSmem<MP>;
+  auto kern = qlora_decode_kernel<MP>;
+  static bool attr_set[kMaxDevices];
+  static int max_clusters[kMaxDevices][9];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    for (int S = 1; S <= 8; ++S) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, 1, static_cast<unsigned>(S));
+      cfg.blockDim = dim3(kDecThreads);
+      cfg.dynamicSmemBytes = L::kDynBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 1;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = static_cast<unsigned>(S);
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      max_clusters[dev][S] = n;
+    }
+    attr_set[dev] = true;
+  }
+  const int T = d.tile_rows;
+  const int tiles = (d.n_cols + T - 1) / T;
+  int S = 1;
+  for (int c = 2; c <= 8; ++c) {
+    const int per = (d.k_steps + c - 1) / c;
+    if (per < 2 || (c - 1) * per >= d.k_steps) continue;   // every rank gets work
+    if (tiles <= max_clusters[dev][c]) S = c;
+  }
+  d.steps_per_split = (d.k_steps + S - 1) / S;
+  d.slice_rows = ((T + S - 1) / S + 7) / 8 * 8;
+  d.slice_u = (d.r + S - 1) / S;
+  if (S * d.slice_rows > 192 || S * d.slice_u > 72) return QLORA_ERR_UNSUPPORTED_SHAPE;  // not reached: r <= 64
+  return timed(QLORA_KERNEL_FWD_DECODE, st, [&] {
+    return launch_ex(kern, dim3(static_cast<unsigned>(tiles), 1, static_cast<unsigned>(S)), dim3(kDecThreads),
+                     L::kDynBytes, st, 1, static_cast<unsigned>(S), tx, tp, ta, tb, d);
+  });
+}
+
+int run_decode(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K, const uint16_t* X,
+               int64_t M, const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* Y, uint16_t* U_save,
+               cudaStream_t st, int dev) {
+  const int mp = M <= 16 ? 16 : 32;
+  const int T = kDecLanes - r;
+  CUtensorMap tx, tp, ta, tb;
+  if (!map_bf16(&tx, X, M, K, 64, static_cast<uint32_t>(mp)) ||
+      !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 32, static_cast<uint32_t>(T),
+                CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !map_bf16(&ta, A, r, K, 64, static_cast<uint32_t>(r)) || !map_bf16(&tb, B, N, r, 64, kDecLanes))
+    return QLORA_ERR_CUDA;
+  DecodeArgs d{};
+  d.m_rows = static_cast<int>(M);
+  d.n_cols = static_cast<int>(N);
+  d.k_steps = static_cast<int>(K / 64);
+  d.steps_per_split = d.k_steps;
+  d.r = r;
+  d.tile_rows = T;
+  d.s = s;
+  d.q8 = q8;
+  d.s2 = s2;
+  for (int i = 0; i < 16; ++i) d.level[i] = tables().level[i];
+  d.y = Y;
+  d.ld_y = N;
+  d.u_save = U_save;
+  if (mp == 16) return launch_decode<16>(tx, tp, ta, tb, d, st, dev);
+  return launch_decode<32>(tx, tp, ta, tb, d, st, dev);
+}
+
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
@@ -507,6 +593,10 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   uint16_t* Us = reinterpret_cast<uint16_t*>(ws + L.us);
   const float s = alpha / static_cast<float>(r);
   const int rpad = (r + 63) / 64 * 64;
+
+  // a few tokens: one launch, weight rows on the MMA's M side, U computed in-kernel
+  if (M <= kDecMaxTokens && r <= kDecMaxRank)
+    return run_decode(codes, q8, s2, n_out, k_in, X, M, A, B, r, s, Y, U_save, st, dev);
 
   if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, sms, st, dev)) return rc;
 

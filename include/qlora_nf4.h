@@ -203,7 +203,8 @@ int qlora_device_status(void* stream);
 #define QLORA_KERNEL_DX 5          /* fused transposed-dequant GEMM: dX       */
 #define QLORA_KERNEL_GRAD_GEMM 6   /* dA^T = X^T V, dB = dY^T U (partials)    */
 #define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
-#define QLORA_KERNEL_COUNT 8
+#define QLORA_KERNEL_FWD_DECODE 8  /* small-M forward (M <= 32, r <= 64)     */
+#define QLORA_KERNEL_COUNT 9
 int qlora_timing_enable(int on);
 /* Number of kernels the library has enqueued since it was loaded (all
  * devices, all streams), counted whether or not timing is enabled. */

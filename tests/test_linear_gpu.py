@@ -117,3 +117,21 @@ def test_adapter_slices_filling_every_stage_back_to_back(M, N, K):
     checks the pipeline's phase handling, not just the arithmetic."""
     for seed in (301, 302):
         run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=256, seed=seed))
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (1, 4096, 4096, 8),      # one token, K split over a cluster
+    (2, 320, 64, 8),         # one k-step (no split), ragged last row tile (320 = 2*128 + 64)
+    (5, 640, 1024, 24),      # rank not a multiple of 16
+    (16, 1024, 640, 64),     # 16 tokens (one 16-token tile), rank 64
+    (17, 384, 2048, 16),     # one past a 16-token tile
+    (32, 256, 4096, 32),
+    (33, 512, 512, 8),       # one past a 32-token tile
+    (64, 768, 1536, 64),     # the largest small-M case
+])
+def test_small_m_forward_and_saved_u(M, N, K, r):
+    """Few-token forward (M <= 32): weight rows and adapter rows share the
+    MMA's row side, the K range is split over a cluster, U = X A^T is formed
+    per K range in the same launch.  M = 33 and 64 cross into the tiled path.
+    Y and the saved U against the oracle; the backward then uses that saved U."""
+    run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=500 + M))
