@@ -214,6 +214,194 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------- decode shapes
+DECODE_N = DECODE_K = 4096
+DECODE_RANK = 8
+DECODE_COPIES = 32          # rotated weight copies: 32 x 8.65 MB = 277 MB, more than L2
+DECODE_REPLAYS = 20
+
+
+def decode_weight_bytes(N, K):
+    """Algorithmic bytes a decode forward must read: packed codes + q8 + s2."""
+    n = N * K
+    nb = n // 64
+    return n // 2 + nb + 4 * ((nb + 255) // 256)
+
+
+def run_decode(q, dev, peaks):
+    """Forward of one 4096 x 4096 NF4+DQ layer (r = 8) at M in {1, 4, 16}: a
+    CUDA graph of 32 layers, each on its own copy of the weight, replayed;
+    time per layer from CUDA events around the replays."""
+    import torch
+    from bit_nf4_quantized_quantize_b200 import synth
+    N, K, r = DECODE_N, DECODE_K, DECODE_RANK
+    inp = synth.layer_inputs("decode", M=16)
+    W = torch.from_numpy(inp["W"]).to(dev)
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(W)
+    copies = [(codes.clone(), q8.clone(), s2.clone()) for _ in range(DECODE_COPIES)]
+    A = torch.from_numpy(inp["A"].view(np.int16)).view(torch.bfloat16).to(dev)
+    B = torch.from_numpy(inp["B"].view(np.int16)).view(torch.bfloat16).to(dev)
+    wbytes = decode_weight_bytes(N, K)
+    out = {}
+    for M in (1, 4, 16):
+        X = torch.from_numpy(inp["X"][:M].view(np.int16)).view(torch.bfloat16).to(dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+
+        def layers():
+            for c in copies:
+                q.qlora_linear_fwd(*c, N, K, X, A, B, inp["alpha"], Y=Y, workspace=ws)
+
+        layers()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                layers()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(DECODE_REPLAYS):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (DECODE_REPLAYS * DECODE_COPIES)
+        gbs = wbytes / (us * 1e-6) / 1e9
+        out[str(M)] = {"us_per_layer": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+        del g
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the decode region: {q.qlora_strerror(rc)}")
+    return {"workload": f"one {N}x{K} NF4+DQ layer, forward, r={r}, alpha=16; CUDA graph of {DECODE_COPIES} layers "
+                        f"on rotated weight copies ({DECODE_COPIES * wbytes / 1e6:.0f} MB, more than L2)",
+            "bound": "hbm", "algorithmic_bytes_per_layer": wbytes, "peak_gbs": peaks["hbm_gbs"],
+            "unit": "GB/s", "by_tokens": out}
+
+
+# ---------------------------------------------------------------------------- larger configurations
+STACK_7B = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]   # q, k, v, o, gate, up, down
+LINEARS_65B = [(8192, 8192), (22016, 8192)]
+STREAM_CHUNKS, STREAM_CHUNK_PARAMS = 30, 1 << 26   # 30 x 256 MiB of fp32 = 2.01e9 parameters
+
+
+def gpu_weight(gen, N, K, kind, dev):
+    """Seeded synthetic weight on the GPU: N(0, 0.02^2), optionally with 0.1% +-6 sigma outliers, or
+    Student-t (4 degrees of freedom) scaled to std 0.02."""
+    import torch
+    if kind == "student_t4":
+        z = torch.randn(N, K, generator=gen, device=dev)
+        chi2 = sum(torch.randn(N, K, generator=gen, device=dev) ** 2 for _ in range(4))
+        return z / torch.sqrt(chi2 / 4) * (0.02 / 2 ** 0.5)
+    w = torch.randn(N, K, generator=gen, device=dev) * 0.02
+    if kind == "normal+outliers":
+        mask = torch.rand(N, K, generator=gen, device=dev) < 1e-3
+        sign = torch.where(torch.rand(N, K, generator=gen, device=dev) < 0.5, -1.0, 1.0)
+        w = torch.where(mask, 0.12 * sign, w)
+    return w
+
+
+def time_region(fn, warmup, reps):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_linear_stack(q, dev, shapes, M, r, alpha, kind, seed, peaks, warmup=2, reps=5):
+    """fwd through every linear, then bwd in reverse order; weights quantized once beforehand."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    layers = []
+    for (N, K) in shapes:
+        W = gpu_weight(gen, N, K, kind, dev)
+        codes, q8, s2 = q.qlora_quantize_nf4_dq(W)
+        del W
+        L = dict(N=N, K=K, codes=codes, q8=q8, s2=s2,
+                 X=torch.randn(M, K, generator=gen, device=dev).bfloat16(),
+                 A=(torch.randn(r, K, generator=gen, device=dev) / K ** 0.5).bfloat16(),
+                 B=(torch.randn(N, r, generator=gen, device=dev) * 0.01).bfloat16(),
+                 dY=torch.randn(M, N, generator=gen, device=dev).bfloat16(),
+                 Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                 U=torch.empty(M, r, dtype=torch.bfloat16, device=dev),
+                 dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+                 dA=torch.empty(r, K, dtype=torch.float32, device=dev),
+                 dB=torch.empty(N, r, dtype=torch.float32, device=dev),
+                 ws=torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev))
+        layers.append(L)
+
+    def step():
+        for L in layers:
+            q.qlora_linear_fwd(L["codes"], L["q8"], L["s2"], L["N"], L["K"], L["X"], L["A"], L["B"], alpha,
+                               Y=L["Y"], U_save=L["U"], workspace=L["ws"])
+        for L in reversed(layers):
+            q.qlora_linear_bwd(L["codes"], L["q8"], L["s2"], L["N"], L["K"], L["X"], L["A"], L["B"], alpha,
+                               L["dY"], U_saved=L["U"], dX=L["dX"], dA=L["dA"], dB=L["dB"], workspace=L["ws"])
+
+    ms = time_region(step, warmup, reps)
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the linear stack: {q.qlora_strerror(rc)}")
+    fl = sum(step_flops(M, N, K, r) for (N, K) in shapes)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"shapes": [f"{N}x{K}" for (N, K) in shapes], "M": M, "r": r, "ms_per_step": ms,
+            "algorithmic_flop": fl, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16"],
+            "steps": reps, "warmup": warmup}
+
+
+def run_quantize_stream(q, dev, peaks, seed=5, reps=3):
+    """NF4 + DQ over 30 chunks of 2^26 Student-t parameters (256 MiB of fp32 each), one launch per chunk."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    n = STREAM_CHUNK_PARAMS
+    W = torch.empty(STREAM_CHUNKS, n, dtype=torch.float32, device=dev)
+    for c in range(STREAM_CHUNKS):
+        W[c] = gpu_weight(gen, 1, n, "student_t4", dev).view(-1)
+    nc, nb, ng = q._binding.quant_sizes(n // 4096, 4096)
+    codes = torch.empty(STREAM_CHUNKS, nc, dtype=torch.uint8, device=dev)
+    q8 = torch.empty(STREAM_CHUNKS, nb, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(STREAM_CHUNKS, ng, dtype=torch.float32, device=dev)
+
+    def one_pass():
+        for c in range(STREAM_CHUNKS):
+            q.qlora_quantize_nf4_dq(W[c].view(n // 4096, 4096), codes[c], q8[c], s2[c])
+
+    ms = time_region(one_pass, 1, reps)
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the quantize stream: {q.qlora_strerror(rc)}")
+    byts = STREAM_CHUNKS * quant_bytes(n // 4096, 4096)
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"params": STREAM_CHUNKS * n, "chunks": STREAM_CHUNKS, "chunk_bytes_fp32": 4 * n, "ms_per_pass": ms,
+            "algorithmic_bytes": byts, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "passes": reps}
+
+
+def run_configs(q, dev, peaks):
+    import torch
+    out = {"data": "seeded synthetic, generated on the GPU (torch generator) with the distributions named "
+                   "per config; weights quantized once, outside the timed region"}
+    out["llama7b_stack"] = run_linear_stack(q, dev, STACK_7B, 2048, 64, 16.0, "normal+outliers", 4, peaks)
+    torch.cuda.empty_cache()
+    out["llama65b_linears"] = run_linear_stack(q, dev, LINEARS_65B, 8192, 64, 16.0, "student_t4", 5, peaks)
+    torch.cuda.empty_cache()
+    out["llama65b_quantize_stream"] = run_quantize_stream(q, dev, peaks)
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------- GPU
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -258,13 +446,23 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     if args.profile:
-        # profiling case for ncu: one step to load the modules, one step to capture
+        # profiling case for ncu: one step to load the modules, one step to
+        # capture, then two decode forwards (M = 1, r = 8) on the same weight.
+        # Launches: [L2 fill + 6 step kernels] x 2, then 2 decode kernels.
+        from bit_nf4_quantized_quantize_b200 import synth
+        dinp = synth.layer_inputs("decode", M=1)
+        decX, decA, decB = (torch.from_numpy(dinp[k].view(np.int16)).view(torch.bfloat16).to(dev)
+                            for k in ("X", "A", "B"))
+        decY = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        dws = torch.empty(q.qlora_workspace_bytes(1, N, K, DECODE_RANK), dtype=torch.uint8, device=dev)
         for i in range(2):
             flush.fill_(float(i))
             step()
+        for _ in range(2):
+            q.qlora_linear_fwd(codes, q8, s2, N, K, decX, decA, decB, dinp["alpha"], Y=decY, workspace=dws)
         torch.cuda.synchronize()
         rc = q.qlora_device_status()
-        print(json.dumps({"profile_case": WORKLOAD, "device_status": rc}), flush=True)
+        print(json.dumps({"profile_case": WORKLOAD + " step + decode M=1", "device_status": rc}), flush=True)
         if rc != 0:
             raise RuntimeError(q.qlora_strerror(rc))
         return
@@ -401,6 +599,9 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "clocks": clocks,
     }
+    line["decode"] = run_decode(q, dev, peaks)
+    if not args.no_configs:
+        line["configs"] = run_configs(q, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp)
     print(json.dumps(line), flush=True)
@@ -413,6 +614,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the 7B-stack / 65B-linear / quantize-stream measurements")
     ap.add_argument("--profile", action="store_true",
                     help="run two steps and exit (the case ncu captures); no timing")
     args = ap.parse_args()
