@@ -71,6 +71,7 @@ def _load():
             lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
             lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.oracle_dequant.argtypes = [P, P, P, i64, P, P, P]
+            lib.oracle_dequant_single.argtypes = [P, P, i64, P, P, P]
             lib.oracle_linear_fwd.argtypes = [P, P, P, P, i64, i64, i64, ctypes.c_int,
                                               ctypes.c_double, P, i64, P, P]
             lib.oracle_linear_bwd.argtypes = [P, P, P, P, P, i64, i64, i64, ctypes.c_int,
@@ -148,6 +149,19 @@ def dequant(codes, q8, s2, n: int, table32: np.ndarray | None = None):
     f32 = np.zeros(n, np.float32)
     b16 = np.zeros(n, np.uint16)
     _load().oracle_dequant(_p(codes), _p(q8), _p(s2), n, _p(t), _p(f32), _p(b16))
+    return f32, b16
+
+
+def dequant_single(codes, absmax, n: int, table32: np.ndarray | None = None):
+    """Single quantization (no second stage): -> (w32 f32[n], w bf16 bits u16[n])."""
+    t = nf4_codebook()[1] if table32 is None else np.ascontiguousarray(table32, np.float32)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    absmax = np.ascontiguousarray(absmax, np.float32)
+    if codes.size * 2 < n or absmax.size * BLOCK < n:
+        raise ValueError("buffers too small for n")
+    f32 = np.zeros(n, np.float32)
+    b16 = np.zeros(n, np.uint16)
+    _load().oracle_dequant_single(_p(codes), _p(absmax), n, _p(t), _p(f32), _p(b16))
     return f32, b16
 
 

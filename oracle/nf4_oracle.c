@@ -27,7 +27,8 @@
  *   - double quantization: linear unsigned 8-bit absmax quantization of each
  *     group of 256 fp32 absmax constants, s2 = fp32(c2/255),
  *     q = min(255, round-half-even(fp32(absmax/s2))), s2 == 0 gives q = 0;
- *   - dequant: w = bf16( fp32( c[code] * fp32(q * s2) ) ).
+ *   - dequant: w = bf16( fp32( c[code] * fp32(q * s2) ) );
+ *   - single quantization (second stage off): w = bf16( fp32( c[code] * absmax ) ).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * fp-contract is off so that no multiply-add is fused: every fp32 operation
@@ -220,6 +221,24 @@ void oracle_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2,
         int code = (i & 1) ? (codes[i / 2] >> 4) : (codes[i / 2] & 15);
         volatile float c1 = (float)q8[b] * s2[g];
         volatile float w32 = table[code] * c1;
+        if (out_f32) out_f32[i] = w32;
+        if (out_bf16) out_bf16[i] = oracle_f32_to_bf16(w32);
+    }
+}
+
+/* Single quantization: only the first stage of p1 §5-2 ("Double
+ * Quantization", memory arithmetic: first stage only = 4 + 32/64 = 4.5
+ * bit/param; the p1 bitsandbytes listing's bnb_4bit_use_double_quant knob
+ * turns the second stage off).  The fp32 absmax of each 64-block is kept as
+ * is, so the block scale is absmax itself:
+ * w = bf16( fp32( c[code] * absmax ) ). */
+void oracle_dequant_single(const uint8_t* codes, const float* absmax, int64_t n,
+                           const float table[16], float* out_f32, uint16_t* out_bf16) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t b = i / ORACLE_BLOCK;
+        int code = (i & 1) ? (codes[i / 2] >> 4) : (codes[i / 2] & 15);
+        volatile float w32 = table[code] * absmax[b];
         if (out_f32) out_f32[i] = w32;
         if (out_bf16) out_bf16[i] = oracle_f32_to_bf16(w32);
     }

@@ -311,6 +311,62 @@ def test_dequant_matches_formula_in_fp32_numpy():
     assert np.max(np.abs(w32 - w)) < 0.2 * np.abs(w).max()
 
 
+# ------------------------------------------------------- single quantization
+def test_single_quant_round_trip_and_size():
+    """First stage only (p1 §5-2 memory arithmetic, Single Q): the block scale is
+    absmax itself, so table values times a power of two come back bit-exactly,
+    and the stored buffers come to the printed 4 + 32/64 = 4.5 bit/param."""
+    _, t32 = oracle.nf4_codebook()
+    blk = np.repeat(t32, 4).astype(np.float32)
+    for e in (-7, 0, 9):
+        x = (blk * np.float32(2.0 ** e)).astype(np.float32)
+        codes, absmax = oracle.quantize_nf4(x)
+        assert absmax[0] == np.float32(2.0 ** e)
+        w32, wb = oracle.dequant_single(codes, absmax, 64)
+        assert np.array_equal(w32.view(np.uint32), x.view(np.uint32))
+        tb = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(wb, tb)
+    w = synth.weight(1, 0, 256, 256).reshape(-1)
+    codes, absmax = oracle.quantize_nf4(w)
+    assert 8 * (codes.nbytes + absmax.nbytes) / w.size == GOLDEN["single_quant_total_bit_per_param"]["value"]
+
+
+def test_single_quant_dequant_formula_and_error_bound():
+    """Independent fp32 restatement in numpy, bf16 against torch, and the
+    reconstruction error within half the widest level gap times absmax."""
+    w = synth.weight(3, 0, 512, 512).reshape(-1)
+    codes, absmax = oracle.quantize_nf4(w)
+    _, t32 = oracle.nf4_codebook()
+    w32, wb = oracle.dequant_single(codes, absmax, w.size)
+    un = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    ref = (t32[un] * np.repeat(absmax, 64)).astype(np.float32)
+    assert np.array_equal(w32.view(np.uint32), ref.view(np.uint32))
+    tb = torch.from_numpy(ref.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(wb, tb)
+    half_gap = np.max(np.diff(t32.astype(np.float64))) / 2
+    err = np.abs(w32.astype(np.float64) - w) / np.repeat(absmax, 64).astype(np.float64)
+    assert np.max(err) <= half_gap * (1 + 1e-6)
+
+
+def test_single_and_double_quant_agree_when_dq_is_exact():
+    """When every absmax of a group equals the group maximum and that maximum is
+    a power of two, fp32(255 * fp32(c2/255)) == c2, so the two-level scale is
+    the absmax itself and both dequantizations give the same bits."""
+    g = np.random.default_rng(11)
+    nblk = 256
+    codes = g.integers(0, 16, size=(nblk, 64))
+    codes[:, 0] = 0                                     # every block holds level -1 -> absmax = scale
+    _, t32 = oracle.nf4_codebook()
+    for e in (-12, 0, 3):
+        sc = np.float32(2.0 ** e)
+        w = (t32[codes] * sc).astype(np.float32).reshape(-1)
+        c, q8, s2, absmax = oracle.quantize_nf4_dq(w)
+        assert np.all(absmax == sc) and np.all(q8 == 255)
+        a, ab = oracle.dequant(c, q8, s2, w.size)
+        b, bb = oracle.dequant_single(c, absmax, w.size)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32)) and np.array_equal(ab, bb)
+
+
 # ----------------------------------------------------------------- linear
 def _small_case(M=9, N=24, K=64, r=3, seed=0):
     g = np.random.default_rng(seed)
