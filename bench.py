@@ -389,6 +389,63 @@ def run_quantize_stream(q, dev, peaks, seed=5, reps=3):
             "algorithmic_bytes": byts, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "passes": reps}
 
 
+def run_single_quant(q, dev, peaks, reps=20):
+    """The train4096 layer with the second quantization stage off: quantize GB/s
+    (4 B read, 0.5 + 4/64 B written per weight) and fwd+bwd TFLOP/s."""
+    import torch
+    N, K, M, r, alpha = N_OUT, K_IN, M_TOK, RANK, ALPHA
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    W = gpu_weight(gen, N, K, "normal", dev)
+    codes = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    qbytes = 4 * N * K + N * K // 2 + 4 * (N * K // 64)
+
+    def quant():
+        flush.fill_(0.0)
+        q.qlora_quantize_nf4(W, codes, absmax)
+
+    # time the quantize launches alone: events around each, after an L2 flush
+    for _ in range(3):
+        quant()
+    ev = []
+    for _ in range(reps):
+        flush.fill_(0.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        q.qlora_quantize_nf4(W, codes, absmax)
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    q_ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    L = dict(X=torch.randn(M, K, generator=gen, device=dev).bfloat16(),
+             A=(torch.randn(r, K, generator=gen, device=dev) / K ** 0.5).bfloat16(),
+             B=(torch.randn(N, r, generator=gen, device=dev) * 0.01).bfloat16(),
+             dY=torch.randn(M, N, generator=gen, device=dev).bfloat16())
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step():
+        q.qlora_linear_fwd(codes, None, absmax, N, K, L["X"], L["A"], L["B"], alpha, Y=Y, U_save=U, workspace=ws)
+        q.qlora_linear_bwd(codes, None, absmax, N, K, L["X"], L["A"], L["B"], alpha, L["dY"], U_saved=U, dX=dX,
+                           dA=dA, dB=dB, workspace=ws)
+
+    ms = time_region(step, 3, 10)
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the single-quantization region: {q.qlora_strerror(rc)}")
+    tf = step_flops(M, N, K, r) / (ms * 1e-3) / 1e12
+    gbs = qbytes / (q_ms * 1e-3) / 1e9
+    return {"workload": "train4096 layer, second quantization stage off (4.5 bit/param)",
+            "quantize_gbs": gbs, "quantize_frac": gbs / peaks["hbm_gbs"], "quantize_algorithmic_bytes": qbytes,
+            "fwd_bwd_tflops": tf, "fwd_bwd_ms": ms}
+
+
 def run_configs(q, dev, peaks):
     import torch
     out = {"data": "seeded synthetic, generated on the GPU (torch generator) with the distributions named "
@@ -398,6 +455,8 @@ def run_configs(q, dev, peaks):
     out["llama65b_linears"] = run_linear_stack(q, dev, LINEARS_65B, 8192, 64, 16.0, "student_t4", 5, peaks)
     torch.cuda.empty_cache()
     out["llama65b_quantize_stream"] = run_quantize_stream(q, dev, peaks)
+    torch.cuda.empty_cache()
+    out["train4096_single_quant"] = run_single_quant(q, dev, peaks)
     torch.cuda.empty_cache()
     return out
 

@@ -26,6 +26,8 @@ _SIGNATURES = {
     "qlora_nf4_codebook": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_quantize_nf4_dq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_quantize_nf4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_dequant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                      ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
@@ -147,12 +149,36 @@ def qlora_quantize_nf4_dq(W, codes=None, q8=None, s2=None, stream=None):
     return codes, q8, s2
 
 
-def qlora_dequant(codes, q8, s2, n_out: int, k_in: int, out=None, dtype=torch.bfloat16, stream=None):
-    """Dense [N, K] dequantized weight (bf16 or fp32)."""
+def _weight(codes, q8, s2, n_out: int, k_in: int):
+    """Check a quantized weight: (codes, q8, s2) with double quantization, or
+    (codes, None, absmax) with single quantization (s2 = fp32 absmax per block)."""
     nc, nb, ng = quant_sizes(n_out, k_in)
     _dev(codes, torch.uint8, "codes", (nc,))
-    _dev(q8, torch.uint8, "q8", (nb,))
-    _dev(s2, torch.float32, "s2", (ng,))
+    if q8 is None:
+        _dev(s2, torch.float32, "absmax", (nb,))
+    else:
+        _dev(q8, torch.uint8, "q8", (nb,))
+        _dev(s2, torch.float32, "s2", (ng,))
+
+
+def qlora_quantize_nf4(W, codes=None, absmax=None, stream=None):
+    """NF4 without the second stage (single quantization) of a fp32 [N, K] CUDA
+    tensor -> (codes, absmax); use (codes, None, absmax) as the weight."""
+    _dev(W, torch.float32, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [n_out, k_in]")
+    N, K = W.shape
+    nc, nb, _ = quant_sizes(N, K)
+    dev = W.device
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev) if codes is None else _dev(codes, torch.uint8, "codes", (nc,))
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev) if absmax is None else _dev(absmax, torch.float32, "absmax", (nb,))
+    _check(load().qlora_quantize_nf4(_ptr(W), N, K, _ptr(codes), _ptr(absmax), _stream(stream)), "qlora_quantize_nf4")
+    return codes, absmax
+
+
+def qlora_dequant(codes, q8, s2, n_out: int, k_in: int, out=None, dtype=torch.bfloat16, stream=None):
+    """Dense [N, K] dequantized weight (bf16 or fp32)."""
+    _weight(codes, q8, s2, n_out, k_in)
     if dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("dtype must be bfloat16 or float32")
     if out is None:
@@ -181,10 +207,7 @@ def _workspace(ws, M, N, K, r, device):
 def qlora_linear_fwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float,
                      Y=None, U_save=None, workspace=None, stream=None):
     """Y = X dequant(W)^T + (alpha/r) (X A^T) B^T in bf16; returns Y (and fills U_save if given)."""
-    nc, nb, ng = quant_sizes(n_out, k_in)
-    _dev(codes, torch.uint8, "codes", (nc,))
-    _dev(q8, torch.uint8, "q8", (nb,))
-    _dev(s2, torch.float32, "s2", (ng,))
+    _weight(codes, q8, s2, n_out, k_in)
     M = X.shape[0]
     r = A.shape[0]
     _dev(X, torch.bfloat16, "X", (M, k_in))
@@ -204,10 +227,7 @@ def qlora_linear_fwd_noalloc(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
                              Y=None, U_save=None, stream=None):
     """qlora_linear_fwd using the library's fixed 4 MiB device scratch (no workspace, no allocation
     inside the library; the binding still allocates Y here if the caller passes none)."""
-    nc, nb, ng = quant_sizes(n_out, k_in)
-    _dev(codes, torch.uint8, "codes", (nc,))
-    _dev(q8, torch.uint8, "q8", (nb,))
-    _dev(s2, torch.float32, "s2", (ng,))
+    _weight(codes, q8, s2, n_out, k_in)
     M = X.shape[0]
     r = A.shape[0]
     _dev(X, torch.bfloat16, "X", (M, k_in))
@@ -225,10 +245,7 @@ def qlora_linear_fwd_noalloc(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
 def qlora_linear_bwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float, dY, U_saved=None,
                      dX=None, dA=None, dB=None, need_dX=True, workspace=None, stream=None):
     """(dX bf16 [M,K] or None, dA fp32 [r,K], dB fp32 [N,r])."""
-    nc, nb, ng = quant_sizes(n_out, k_in)
-    _dev(codes, torch.uint8, "codes", (nc,))
-    _dev(q8, torch.uint8, "q8", (nb,))
-    _dev(s2, torch.float32, "s2", (ng,))
+    _weight(codes, q8, s2, n_out, k_in)
     M = X.shape[0]
     r = A.shape[0]
     _dev(X, torch.bfloat16, "X", (M, k_in))

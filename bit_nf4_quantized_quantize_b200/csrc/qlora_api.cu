@@ -438,8 +438,10 @@ LoraProblem lora_problem(int rows, int k_steps, int S, int rpad, int kind, void*
   return p;
 }
 
+// q8 == NULL: single quantization, s2 holds the fp32 absmax of every block.
 int check_weight(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K) {
-  if (!codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
+  (void)q8;
+  if (!codes || !s2) return QLORA_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || K % 64 != 0 || N % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (N > (1 << 24) || K > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(codes) || !aligned16(s2)) return QLORA_ERR_UNSUPPORTED_SHAPE;
@@ -544,14 +546,32 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_dq_kernel, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1, 1, W,
-                     n_blocks, codes, q8, s2, tables());
+    return launch_ex(quantize_nf4_kernel<true>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
+                     1, W, n_blocks, codes, q8, s2, tables());
+  });
+}
+
+int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, float* absmax, void* stream) {
+  if (!W || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
+  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(absmax) & 3u))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const int64_t n_blocks = n_out * k_in / kBlock;
+  const int64_t groups = (n_blocks + kGroup - 1) / kGroup;
+  if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* no_q8 = nullptr;
+  return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
+    return launch_ex(quantize_nf4_kernel<false>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
+                     1, W, n_blocks, codes, no_q8, absmax, tables());
   });
 }
 
 int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
                   void* out, int out_dtype, void* stream) {
-  if (!codes || !q8 || !s2 || !out) return QLORA_ERR_INVALID_ARG;
+  if (!codes || !s2 || !out) return QLORA_ERR_INVALID_ARG;   // q8 == NULL: single quantization
   if (out_dtype != QLORA_OUT_BF16 && out_dtype != QLORA_OUT_FP32) return QLORA_ERR_INVALID_ARG;
   if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if ((reinterpret_cast<uintptr_t>(codes) & 3u) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;

@@ -2,15 +2,17 @@
 //
 // "QLoRAの理論と実装" §5-1 (absmax per 64-block, w/absmax, nearest of the 16
 // NormalFloat levels, 4-bit code) and §5-2 (8-bit re-quantization of the fp32
-// absmax constants in groups of 256, one fp32 second-level constant).
+// absmax constants in groups of 256, one fp32 second-level constant; without
+// that second stage the fp32 absmax constants are stored as they are).
 //
-// quantize_dq_kernel: one CTA of 512 threads per group of 256 blocks (16384
+// quantize_nf4_kernel<kDQ>: one CTA of 512 threads per group of 256 blocks (16384
 // weights, 64 KiB of fp32 input).  Eight threads share a 64-block (8
 // consecutive weights each, two 16-byte loads), so a warp reads 1 KiB
 // contiguous per pass; the block absmax is a 3-step xor-shuffle max.  The
 // group's 256 absmax values then stay in shared memory for the second-level
 // quantization, so the fp32 constants never go to HBM.  Traffic per weight:
-// 4 B read, 0.5 + 1/64 + 4/16384 B written.
+// 4 B read, 0.5 + 1/64 + 4/16384 B written (kDQ), or 0.5 + 4/64 B written
+// when the second stage is off and the absmax constants are stored.
 //
 // Nearest level.  The code of n = fp32(w / absmax) is #{i : n >= thr_i}, thr_i
 // the smallest fp32 above the exact midpoint of levels i and i+1.  Cells of
@@ -48,9 +50,12 @@ struct Nf4Tables {
 
 constexpr int kQuantThreads = 512;  // 16 warps; 8 threads per 64-block, 4 passes of 64 blocks
 
+// kDQ: q8 / s2 receive the second-level quantization of the absmax constants.
+// !kDQ: q8 is unused and s2 receives the n_blocks fp32 absmax constants.
+template <bool kDQ>
 __global__ void __launch_bounds__(kQuantThreads, 2)
-quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
-                   uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
+quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
+                    uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
   __shared__ int2 s_exact[kLutCells];     // {threshold bits, left-edge code}
   __shared__ uint32_t s_fast[kLutCells];
   __shared__ float s_absmax[kGroup];
@@ -128,10 +133,14 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
         packed |= static_cast<uint32_t>(code) << (4 * j);
       }
       *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
-      if (sub == 0) s_absmax[lb] = am;
+      if (sub == 0) {
+        if (kDQ) s_absmax[lb] = am;
+        else s2[b_first + lb] = am;
+      }
     }
   }
   griddep_launch_dependents();
+  if (!kDQ) return;
   __syncthreads();
 
   // Second level: c2 = max of the group's absmax, s2 = fp32(c2/255),
@@ -162,8 +171,10 @@ quantize_dq_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __res
   }
 }
 
-// Dense dequantization: w = fp32(level[code] * fp32(q * s2)), fp32 or bf16 out.
-// One thread per 8 consecutive weights (4 packed bytes).
+// Dense dequantization: w = fp32(level[code] * fp32(q * s2)), fp32 or bf16 out;
+// with q8 == nullptr (single quantization) s2 holds the fp32 absmax per block
+// and w = fp32(level[code] * absmax).  One thread per 8 consecutive weights
+// (4 packed bytes).
 template <bool kBf16>
 __global__ void __launch_bounds__(256)
 dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8,
@@ -177,7 +188,8 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(codes) + i);
     const int64_t blk = (i * 8) / kBlock;
-    const float c1 = __fmul_rn(static_cast<float>(__ldg(q8 + blk)), __ldg(s2 + blk / kGroup));
+    const float c1 = q8 == nullptr ? __ldg(s2 + blk)
+                                   : __fmul_rn(static_cast<float>(__ldg(q8 + blk)), __ldg(s2 + blk / kGroup));
     float w[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(s_level[(p >> (4 * j)) & 15u], c1);

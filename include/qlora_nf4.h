@@ -24,13 +24,17 @@
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Every call is asynchronous on that stream: it validates its arguments on
  *   the host, enqueues kernels and returns.
- * - The quantized weight is three flat buffers:
+ * - The quantized weight is three flat buffers (double quantization):
  *     codes  uint8_t[N*K/2]      NF4 codes, row-major, element 2j in the low
  *                                nibble of byte j;
  *     q8     uint8_t[N*K/64]     8-bit absmax constant of each 64-block;
  *     s2     float[ceil(N*K/16384)]  fp32 second-level constant of each group
- *                                of 256 consecutive blocks.
- *   Fixed by the method: block 64, group 256, double quantization on.
+ *                                of 256 consecutive blocks;
+ *   or, with single quantization (the second stage off, 4.5 bit/param), two:
+ *     codes  as above;  q8 = NULL;
+ *     s2     float[N*K/64]       the fp32 absmax constant of each 64-block.
+ *   Every call that takes (codes, q8, s2) reads q8 == NULL as single
+ *   quantization.  Fixed by the method: block 64, group 256.
  * - Preconditions checked on the host (QLORA_ERR_* on violation, nothing
  *   enqueued): non-NULL required pointers, every pointer 16-byte aligned,
  *   K % 64 == 0, N % 64 == 0, M >= 1, 1 <= r <= 256 with r % 8 == 0, alpha
@@ -91,8 +95,24 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in,
                           uint8_t* codes, uint8_t* q8, float* s2, void* stream);
 
 /*
+ * Blockwise NF4 quantization without the second stage (single quantization):
+ * "QLoRAの理論と実装" §5-1 steps 1-2 alone; §5-2's memory arithmetic prices it
+ * at 4 + 32/64 = 4.5 bit/param, and the page's bitsandbytes listing selects it
+ * with bnb_4bit_use_double_quant=False.
+ *
+ *   W       fp32[N*K] device, row-major, read only.
+ *   codes   uint8_t[N*K/2] written (identical to qlora_quantize_nf4_dq's).
+ *   absmax  float[N*K/64]  written: max|w| of each 64-block, exact.
+ * Pass (codes, NULL, absmax) to the dequantization and linear-layer calls.
+ * One kernel launch.
+ */
+int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in,
+                       uint8_t* codes, float* absmax, void* stream);
+
+/*
  * Dequantization to a dense N x K matrix ("QLoRAの理論と実装" §5-1 step 3 with
- * the two-level constant):  w = fp32(level[code] * fp32(q8 * s2)), written as
+ * the two-level constant):  w = fp32(level[code] * fp32(q8 * s2)), or with
+ * q8 == NULL w = fp32(level[code] * absmax) (s2 = absmax), written as
  * fp32 (out_dtype QLORA_OUT_FP32) or rounded to nearest-even bf16
  * (QLORA_OUT_BF16).  `out` is device memory of N*K elements.  This is for
  * tests and export; the linear layer never materialises it.

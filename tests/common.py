@@ -36,3 +36,11 @@ def oracle_weight(W: np.ndarray):
     codes, q8, s2, _ = oracle.quantize_nf4_dq(W.reshape(-1))
     _, wb = oracle.dequant(codes, q8, s2, N * K)
     return codes, q8, s2, bits_f64(wb).reshape(N, K)
+
+
+def oracle_weight_single(W: np.ndarray):
+    """Oracle single quantization + dequant -> (codes, absmax, What bf16 as f64 N x K)."""
+    N, K = W.shape
+    codes, absmax = oracle.quantize_nf4(W.reshape(-1))
+    _, wb = oracle.dequant_single(codes, absmax, N * K)
+    return codes, absmax, bits_f64(wb).reshape(N, K)

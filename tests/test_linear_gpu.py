@@ -15,15 +15,19 @@ import torch
 import oracle
 import bit_nf4_quantized_quantize_b200 as q
 from bit_nf4_quantized_quantize_b200 import synth
-from common import REL_L2_TOL, bf16_to_np_f64, bits_f64, oracle_weight, rel_l2, to_dev_bf16
+from common import REL_L2_TOL, bf16_to_np_f64, bits_f64, oracle_weight, oracle_weight_single, rel_l2, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
 
-def run_case(inp, rows=None, check_bwd=True, dy_rows=None):
+def run_case(inp, rows=None, check_bwd=True, dy_rows=None, single=False):
     N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
     Wd = torch.from_numpy(inp["W"]).cuda()
-    codes, q8, s2 = q.qlora_quantize_nf4_dq(Wd)
+    if single:
+        codes, s2 = q.qlora_quantize_nf4(Wd)   # second stage off: s2 = fp32 absmax
+        q8 = None
+    else:
+        codes, q8, s2 = q.qlora_quantize_nf4_dq(Wd)
     X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
     U = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
     Y = q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, U_save=U)
@@ -33,7 +37,7 @@ def run_case(inp, rows=None, check_bwd=True, dy_rows=None):
         res.update(dX=dX, dA=dA, dB=dB)
     assert q.qlora_device_status() == 0
     # oracle on the same inputs
-    _, _, _, What = oracle_weight(inp["W"])
+    What = oracle_weight_single(inp["W"])[2] if single else oracle_weight(inp["W"])[3]
     Xo, Ao, Bo, dYo = (bits_f64(inp[k]) for k in ("X", "A", "B", "dY"))
     Yr, Ur = oracle.linear_fwd(Xo, What, Ao, Bo, alpha, rows=rows)
     sel = slice(None) if rows is None else rows
@@ -135,3 +139,14 @@ def test_small_m_forward_and_saved_u(M, N, K, r):
     per K range in the same launch.  M = 33 and 64 cross into the tiled path.
     Y and the saved U against the oracle; the backward then uses that saved U."""
     run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=500 + M))
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (1, 4096, 4096, 8),      # few-token path
+    (40, 512, 768, 8),       # tiled path, one CTA per tile
+    (300, 512, 768, 64),     # CTA-pair path
+])
+def test_single_quantization_linear(M, N, K, r):
+    """The layer on a weight without the second quantization stage (q8 = NULL,
+    s2 = fp32 absmax per block): forward and backward against the oracle."""
+    run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=700 + M), single=True)

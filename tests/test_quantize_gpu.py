@@ -50,7 +50,27 @@ def test_ragged_last_group_exact():
     check_exact(synth.weight(12, 0, 1, 64))          # a single block
 
 
-def test_edge_case_blocks_exact():
+def check_exact_single(W: np.ndarray, dequant=True):
+    """Single quantization (second stage off): codes and the fp32 absmax bit-exact,
+    codes identical to the double-quant call's, dense dequant bit-exact."""
+    N, K = W.shape
+    Wd = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    codes, absmax = q.qlora_quantize_nf4(Wd)
+    codes_dq, _, _ = q.qlora_quantize_nf4_dq(Wd)
+    rc, ra = oracle.quantize_nf4(W.reshape(-1))
+    gc, ga = codes.cpu().numpy(), absmax.cpu().numpy()
+    assert np.array_equal(gc, rc)
+    assert np.array_equal(ga.view(np.uint32), ra.view(np.uint32))
+    assert torch.equal(codes, codes_dq)
+    if dequant:
+        w32, wb = oracle.dequant_single(rc, ra, N * K)
+        d32 = q.qlora_dequant(codes, None, absmax, N, K, dtype=torch.float32).cpu().numpy().reshape(-1)
+        db = q.qlora_dequant(codes, None, absmax, N, K, dtype=torch.bfloat16).view(torch.int16).cpu().numpy()
+        assert np.array_equal(d32.view(np.uint32), w32.view(np.uint32))
+        assert np.array_equal(db.reshape(-1).view(np.uint16), wb)
+
+
+def edge_case_weight():
     _, t32 = oracle.nf4_codebook()
     blocks = []
     blocks.append(np.zeros(64, np.float32))                                     # all zero
@@ -84,8 +104,19 @@ def test_edge_case_blocks_exact():
         b[:chunk.size] = chunk
         b[63] = -1.0
         blocks.append(b)
-    W = np.concatenate(blocks).reshape(1, -1)
-    check_exact(W)
+    return np.concatenate(blocks).reshape(1, -1)
+
+
+def test_edge_case_blocks_exact():
+    check_exact(edge_case_weight())
+
+
+def test_single_quant_exact():
+    check_exact_single(synth.weight(1, 0, 256, 256))
+    check_exact_single(synth.weight(11, 0, 3, 6400))           # ragged last group of blocks
+    check_exact_single(edge_case_weight())
+    check_exact_single(synth.weight(3, 0, 4096, 4096))
+    check_exact_single(synth.weight(5, 0, 512, 8192, "student_t4"))
 
 
 def test_all_fp32_near_every_threshold_exact():
