@@ -72,6 +72,9 @@ def _load():
             lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.oracle_dequant.argtypes = [P, P, P, i64, P, P, P]
             lib.oracle_dequant_single.argtypes = [P, P, i64, P, P, P]
+            lib.oracle_f64_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
+            lib.oracle_merge_adapter.argtypes = [P, i64, i64, P, P, ctypes.c_int, ctypes.c_double, P]
             lib.oracle_linear_fwd.argtypes = [P, P, P, P, i64, i64, i64, ctypes.c_int,
                                               ctypes.c_double, P, i64, P, P]
             lib.oracle_linear_bwd.argtypes = [P, P, P, P, P, i64, i64, i64, ctypes.c_int,
@@ -163,6 +166,27 @@ def dequant_single(codes, absmax, n: int, table32: np.ndarray | None = None):
     b16 = np.zeros(n, np.uint16)
     _load().oracle_dequant_single(_p(codes), _p(absmax), n, _p(t), _p(f32), _p(b16))
     return f32, b16
+
+
+def f64_to_bf16_bits(x) -> np.ndarray:
+    """Round fp64 to bf16 (nearest, ties to even) in one step with the oracle's C routine."""
+    x = np.ascontiguousarray(x, np.float64).reshape(-1)
+    f = _load().oracle_f64_to_bf16
+    return np.array([f(float(v)) for v in x], np.uint16)
+
+
+def merge_adapter(W: np.ndarray, A_bits: np.ndarray, B_bits: np.ndarray, alpha: float) -> np.ndarray:
+    """bf16 bits of bf16(bf16(W) + s B A) for fp32 W [N, K], bf16-bit A [r, K], B [N, r]."""
+    W = np.ascontiguousarray(W, np.float32)
+    N, K = W.shape
+    A_bits = np.ascontiguousarray(A_bits, np.uint16)
+    B_bits = np.ascontiguousarray(B_bits, np.uint16)
+    r = A_bits.shape[0]
+    if A_bits.shape != (r, K) or B_bits.shape != (N, r):
+        raise ValueError("A must be r x K and B N x r")
+    out = np.zeros((N, K), np.uint16)
+    _load().oracle_merge_adapter(_p(W), N, K, _p(A_bits), _p(B_bits), r, float(alpha), _p(out))
+    return out
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -10,6 +10,8 @@
  * Every step is written to be read against the pages:
  *   [p1] "QLoRAの理論と実装" (disassemble-channel.com)
  *   [p2] Qiita article on why QLoRA survives 4-bit (TaiyoYamada)
+ *   [p4] "QLoRAとは？4bit量子化＋LoRAの仕組み・VRAM目安・実装手順と採用判断を解説"
+ *        (issoh.co.jp)
  * Quantisation follows the algorithm's steps in order (it is an encoding, so
  * there is no shorter closed form); the linear layer is the plain definition
  * evaluated in fp64 on the exact bf16 operands.
@@ -28,7 +30,9 @@
  *     group of 256 fp32 absmax constants, s2 = fp32(c2/255),
  *     q = min(255, round-half-even(fp32(absmax/s2))), s2 == 0 gives q = 0;
  *   - dequant: w = bf16( fp32( c[code] * fp32(q * s2) ) );
- *   - single quantization (second stage off): w = bf16( fp32( c[code] * absmax ) ).
+ *   - single quantization (second stage off): w = bf16( fp32( c[code] * absmax ) );
+ *   - adapter merge: into the 16-bit base, not the 4-bit one (p4), as one
+ *     rounding of the fp64 value bf16(W) + s * sum_j B[n,j] A[j,k].
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * fp-contract is off so that no multiply-add is fused: every fp32 operation
@@ -241,6 +245,61 @@ void oracle_dequant_single(const uint8_t* codes, const float* absmax, int64_t n,
         volatile float w32 = table[code] * absmax[b];
         if (out_f32) out_f32[i] = w32;
         if (out_bf16) out_bf16[i] = oracle_f32_to_bf16(w32);
+    }
+}
+
+/* fp64 -> bf16, round to nearest, ties to even, in one step (no detour     */
+/* through fp32).  Finite input; values past the largest bf16 become inf.   */
+uint16_t oracle_f64_to_bf16(double x) {
+    if (x == 0.0) return signbit(x) ? 0x8000u : 0x0000u;
+    double a = fabs(x);
+    int e;
+    frexp(a, &e);                        /* a = m * 2^e, 0.5 <= m < 1          */
+    int ue = e - 8;                      /* bf16 keeps 8 significant bits       */
+    if (ue < -133) ue = -133;            /* subnormal bf16: ulp 2^-133          */
+    double q = rint(ldexp(a, -ue));      /* exact scaling, then round-half-even */
+    double r = ldexp(q, ue);             /* exactly representable in fp32       */
+    float f = (float)r;
+    if (r > 3.3895313892515355e38) f = INFINITY;   /* beyond the largest bf16 */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint16_t b = (uint16_t)(u >> 16);
+    return x < 0 ? (uint16_t)(b | 0x8000u) : b;
+}
+
+static double oracle_bf16_to_f64(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Adapter merge for distribution, [p4] "学習済みアダプタのマージと配布で精度が */
+/* 崩れる分岐点を整理する": merging into the 4-bit base rounds the adapter's    */
+/* small differences onto the 4-bit grid, so the adapter is folded into the  */
+/* unquantized base loaded in bf16, and the merged 16-bit weight is then     */
+/* quantized again.  Here: W16 = bf16(W); each output element is            */
+/*   v = fp64(W16) + fp64(s) * sum_{j=0..r-1} B[n,j] A[j,k]                  */
+/* with the sum taken in fp64 in the order j = 0, 1, ..., one rounding per   */
+/* product and per addition (products of two bf16 values are exact in fp64), */
+/* and merged = bf16(v), rounded once.  s = fp32(alpha / r).  W is N x K     */
+/* fp32, A is r x K and B is N x r as bf16 bit patterns; out is N x K bf16.  */
+void oracle_merge_adapter(const float* W, int64_t N, int64_t K, const uint16_t* A, const uint16_t* B,
+                          int r, double alpha, uint16_t* out) {
+    volatile float s32 = (float)(alpha / (double)r);
+    double s = (double)s32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            volatile double acc = 0.0;
+            for (int j = 0; j < r; ++j) {
+                volatile double prod = oracle_bf16_to_f64(B[n * r + j]) * oracle_bf16_to_f64(A[(int64_t)j * K + k]);
+                acc = acc + prod;
+            }
+            volatile double t = s * acc;
+            volatile double v = oracle_bf16_to_f64(oracle_f32_to_bf16(W[n * K + k])) + t;
+            out[n * K + k] = oracle_f64_to_bf16(v);
+        }
     }
 }
 

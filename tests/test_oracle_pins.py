@@ -367,6 +367,94 @@ def test_single_and_double_quant_agree_when_dq_is_exact():
         assert np.array_equal(a.view(np.uint32), b.view(np.uint32)) and np.array_equal(ab, bb)
 
 
+# ---------------------------------------------------------- adapter merge
+def _bf16_exact_nearest(x: float) -> int:
+    """bf16 bits nearest to x (ties to even), by exact rational comparison of the
+    two bf16 neighbours of x (finite bf16 range)."""
+    from fractions import Fraction
+    fx = Fraction(x)
+    if fx == 0:
+        return 0x8000 if np.signbit(x) else 0
+    sign = 0x8000 if fx < 0 else 0
+    a = abs(fx)
+    # candidates: every bf16 magnitude whose fp32 value brackets a
+    lo_bits = int(np.array([np.float32(float(a))], np.float32).view(np.uint32)[0]) >> 16
+    cands = [b for b in (lo_bits - 1, lo_bits, lo_bits + 1, lo_bits + 2) if 0 <= b < 0x7F80]
+    val = lambda b: Fraction(float(np.array([b << 16], np.uint32).view(np.float32)[0]))
+    best = min(cands, key=lambda b: (abs(val(b) - a), b & 1))
+    return sign | best
+
+
+def test_f64_to_bf16_is_nearest_ties_to_even():
+    g = np.random.default_rng(21)
+    xs = list(g.normal(0, 1, 3000)) + list(g.normal(0, 1e-30, 300)) + list(g.normal(0, 1e30, 300))
+    # exact ties between two bf16 values, and points one fp64 ulp either side
+    for b in g.integers(0x0080, 0x7F00, 300):
+        lo = float(np.array([int(b) << 16], np.uint32).view(np.float32)[0])
+        hi = float(np.array([(int(b) + 1) << 16], np.uint32).view(np.float32)[0])
+        mid = (lo + hi) / 2
+        xs += [mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf), -mid]
+    xs = np.array(xs, np.float64)
+    ours = oracle.f64_to_bf16_bits(xs)
+    ref = np.array([_bf16_exact_nearest(float(x)) for x in xs], np.uint16)
+    assert np.array_equal(ours, ref)
+    # fp32-exact inputs agree with torch's fp32 -> bf16 rounding
+    x32 = g.normal(0, 1, 2000).astype(np.float32)
+    tb = torch.from_numpy(x32.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16_bits(x32.astype(np.float64)), tb)
+
+
+def _bf16_bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bits_to_f64(b):
+    return (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_merge_adapter_zero_b_is_the_bf16_base():
+    """[p4] merge into the 16-bit base: with B = 0 the merged weight is bf16(W)."""
+    W = synth.weight(1, 0, 64, 128)
+    A = _bf16_bits(np.random.default_rng(1).normal(0, 0.1, (8, 128)))
+    B = np.zeros((64, 8), np.uint16)
+    assert np.array_equal(oracle.merge_adapter(W, A, B, 16.0), _bf16_bits(W))
+
+
+def test_merge_adapter_exact_rational_cases():
+    """Dyadic inputs of moderate range keep every fp64 step exact, so the merged
+    weight is the exact value bf16(W) + s B A rounded once (Fraction arithmetic)."""
+    from fractions import Fraction
+    g = np.random.default_rng(5)
+    N, K, r, alpha = 12, 40, 4, 16.0              # s = 4, a power of two
+    W = (g.integers(-64, 65, (N, K)) / 64.0).astype(np.float32)
+    A = _bf16_bits(g.integers(-32, 33, (r, K)) / 128.0)
+    B = _bf16_bits(g.integers(-32, 33, (N, r)) / 1024.0)
+    out = oracle.merge_adapter(W, A, B, alpha)
+    Af, Bf = _bits_to_f64(A), _bits_to_f64(B)
+    s = Fraction(alpha) / r
+    for n in range(N):
+        for k in range(K):
+            v = Fraction(float(W[n, k])) + s * sum(Fraction(Bf[n, j]) * Fraction(Af[j, k]) for j in range(r))
+            assert out[n, k] == _bf16_exact_nearest(float(v)), (n, k)
+
+
+def test_merge_adapter_layer_identity():
+    """X merged^T equals X bf16(W)^T + s (X A^T) B^T up to the one bf16 rounding of the merge."""
+    g = np.random.default_rng(8)
+    N, K, M, r, alpha = 96, 192, 5, 8, 16.0
+    W = synth.weight(2, 0, N, K)
+    Ab = _bf16_bits(g.normal(0, 1 / np.sqrt(K), (r, K)))
+    Bb = _bf16_bits(g.normal(0, 0.5, (N, r)))
+    Wm = _bits_to_f64(oracle.merge_adapter(W, Ab, Bb, alpha))
+    X = g.normal(size=(M, K))
+    s = np.float64(np.float32(alpha / r))
+    ref = X @ _bits_to_f64(_bf16_bits(W)).T + s * (X @ _bits_to_f64(Ab).T) @ _bits_to_f64(Bb).T
+    got = X @ Wm.T
+    # each merged element is within half a bf16 ulp (2^-9 relative) of its exact value
+    bound = np.abs(X) @ (np.abs(Wm).T * 2.0 ** -8)
+    assert np.all(np.abs(got - ref) <= bound + 1e-12)
+
+
 # ----------------------------------------------------------------- linear
 def _small_case(M=9, N=24, K=64, r=3, seed=0):
     g = np.random.default_rng(seed)
