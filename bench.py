@@ -446,6 +446,31 @@ def run_single_quant(q, dev, peaks, reps=20):
             "fwd_bwd_tflops": tf, "fwd_bwd_ms": ms}
 
 
+def run_merge(q, dev, peaks, reps=10):
+    """Adapter merge into the bf16 base of the train4096 layer (r = 64), then NF4 + DQ of the
+    merged weight: time of each launch; the merge is fp64-issue bound (2 r fp64 ops per weight)."""
+    import torch
+    N, K, r, alpha = N_OUT, K_IN, RANK, ALPHA
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    W = gpu_weight(gen, N, K, "normal", dev)
+    A = (torch.randn(r, K, generator=gen, device=dev) / K ** 0.5).bfloat16()
+    B = (torch.randn(N, r, generator=gen, device=dev) * 0.01).bfloat16()
+    merged = torch.empty(N, K, dtype=torch.float32, device=dev)
+    codes = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
+    q8 = torch.empty(N * K // 64, dtype=torch.uint8, device=dev)
+    s2 = torch.empty((N * K // 64 + 255) // 256, dtype=torch.float32, device=dev)
+    m_ms = time_region(lambda: q.qlora_merge_adapter(W, A, B, alpha, out=merged), 2, reps)
+    q_ms = time_region(lambda: q.qlora_quantize_nf4_dq(merged, codes, q8, s2), 2, reps)
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the merge region: {q.qlora_strerror(rc)}")
+    fp64_ops = 2 * N * K * r
+    return {"workload": "train4096 layer, r=64: merge into the bf16 base, then NF4+DQ of the merged weight",
+            "merge_ms": m_ms, "merge_fp64_ops": fp64_ops, "merge_fp64_gops_per_s": fp64_ops / (m_ms * 1e-3) / 1e9,
+            "requantize_ms": q_ms, "requantize_gbs": quant_bytes(N, K) / (q_ms * 1e-3) / 1e9}
+
+
 def run_configs(q, dev, peaks):
     import torch
     out = {"data": "seeded synthetic, generated on the GPU (torch generator) with the distributions named "
@@ -457,6 +482,8 @@ def run_configs(q, dev, peaks):
     out["llama65b_quantize_stream"] = run_quantize_stream(q, dev, peaks)
     torch.cuda.empty_cache()
     out["train4096_single_quant"] = run_single_quant(q, dev, peaks)
+    torch.cuda.empty_cache()
+    out["train4096_merge_requantize"] = run_merge(q, dev, peaks)
     torch.cuda.empty_cache()
     return out
 

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     qlora_linear_bwd,
     qlora_linear_fwd,
     qlora_linear_fwd_noalloc,
+    qlora_merge_adapter,
     qlora_nf4_codebook,
     qlora_quantize_nf4_dq,
     qlora_quantize_nf4,

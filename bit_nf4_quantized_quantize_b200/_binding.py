@@ -28,6 +28,9 @@ _SIGNATURES = {
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_quantize_nf4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_merge_adapter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                           ctypes.c_int, ctypes.c_void_p]),
     "qlora_dequant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                      ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
@@ -51,7 +54,7 @@ _SIGNATURES = {
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "lora_gemm", "lora_reduce", "fwd_fused", "dx_fused", "grad_gemm",
-                "grad_reduce", "fwd_decode"]
+                "grad_reduce", "fwd_decode", "merge"]
 
 
 class QloraError(RuntimeError):
@@ -188,6 +191,25 @@ def qlora_dequant(codes, q8, s2, n_out: int, k_in: int, out=None, dtype=torch.bf
     code = QLORA_OUT_BF16 if dtype == torch.bfloat16 else QLORA_OUT_FP32
     _check(load().qlora_dequant(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(out), code, _stream(stream)),
            "qlora_dequant")
+    return out
+
+
+def qlora_merge_adapter(W, A, B, alpha: float, out=None, dtype=torch.float32, stream=None):
+    """Merged 16-bit weight bf16(bf16(W) + (alpha/r) B A) of the fp32 base W [N, K] and the
+    adapter A [r, K], B [N, r] (bf16); fp32 output (bf16 values) feeds re-quantization."""
+    _dev(W, torch.float32, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [n_out, k_in]")
+    N, K = W.shape
+    r = A.shape[0]
+    _dev(A, torch.bfloat16, "A", (r, K))
+    _dev(B, torch.bfloat16, "B", (N, r))
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("dtype must be bfloat16 or float32")
+    out = torch.empty(N, K, dtype=dtype, device=W.device) if out is None else _dev(out, dtype, "out", (N, K))
+    code = QLORA_OUT_BF16 if dtype == torch.bfloat16 else QLORA_OUT_FP32
+    _check(load().qlora_merge_adapter(_ptr(W), N, K, _ptr(A), _ptr(B), r, float(alpha), _ptr(out), code,
+                                      _stream(stream)), "qlora_merge_adapter")
     return out
 
 

@@ -23,6 +23,7 @@
 #include "lora_tc.cuh"
 #include "fused2_tc.cuh"
 #include "decode_tc.cuh"
+#include "merge.cuh"
 
 using namespace qlora;
 
@@ -566,6 +567,31 @@ int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* cod
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
     return launch_ex(quantize_nf4_kernel<false>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
                      1, W, n_blocks, codes, no_q8, absmax, tables());
+  });
+}
+
+int qlora_merge_adapter(const float* W, int64_t n_out, int64_t k_in, const uint16_t* A, const uint16_t* B, int r,
+                        float alpha, void* out, int out_dtype, void* stream) {
+  if (!W || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != QLORA_OUT_BF16 && out_dtype != QLORA_OUT_FP32) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0 || n_out > (1 << 24) || k_in > (1 << 24))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const double s = static_cast<double>(alpha / static_cast<float>(r));
+  if ((n_out + kMergeRows - 1) / kMergeRows > 65535) return QLORA_ERR_UNSUPPORTED_SHAPE;   // grid y
+  const dim3 grid(static_cast<unsigned>((k_in + kMergeCols - 1) / kMergeCols),
+                  static_cast<unsigned>((n_out + kMergeRows - 1) / kMergeRows));
+  const size_t smem = sizeof(double) * kMergeRows * static_cast<size_t>(r);   // <= 32 KiB
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return timed(QLORA_KERNEL_MERGE, st, [&] {
+    if (out_dtype == QLORA_OUT_BF16)
+      return launch_ex(merge_adapter_kernel<true>, grid, dim3(kMergeCols), smem, st, 1, 1, W, n_out, k_in, A, B, r,
+                       s, out);
+    return launch_ex(merge_adapter_kernel<false>, grid, dim3(kMergeCols), smem, st, 1, 1, W, n_out, k_in, A, B, r,
+                     s, out);
   });
 }
 

@@ -121,6 +121,28 @@ int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2,
                   int64_t n_out, int64_t k_in, void* out, int out_dtype,
                   void* stream);
 
+/*
+ * Adapter merge for distribution ("QLoRAとは？4bit量子化＋LoRAの仕組み・VRAM
+ * 目安・実装手順と採用判断を解説", section on merging a trained adapter):
+ * merging onto the 4-bit base rounds the adapter's small differences onto the
+ * 4-bit grid, so the adapter is folded into the unquantized base in bf16 and
+ * the merged 16-bit weight is quantized again.  Per element:
+ *   merged = bf16( fp64(bf16(W)) + fp64(s) * sum_{j=0..r-1} B[n,j] A[j,k] ),
+ * the sum in fp64 in that order (each product and addition rounded once,
+ * no fused multiply-add), one rounding to bf16 at the end; s = fp32(alpha/r).
+ *
+ *   W    fp32[N*K] device, the original (unquantized) weight, read only.
+ *   A    bf16[r*K], B bf16[N*r] device (the trained adapter), read only.
+ *   out  N*K elements: bf16 bits (QLORA_OUT_BF16), or the same bf16 values as
+ *        fp32 (QLORA_OUT_FP32), which qlora_quantize_nf4_dq / qlora_quantize_nf4
+ *        take directly to re-quantize.
+ * 1 <= r <= 256, alpha finite, K % 64 == 0, N <= 1048560, every pointer 16-byte
+ * aligned.  One kernel launch.  There is no counterpart that merges into the NF4
+ * weight: that is the lossy path the page warns against.
+ */
+int qlora_merge_adapter(const float* W, int64_t n_out, int64_t k_in, const uint16_t* A, const uint16_t* B, int r,
+                        float alpha, void* out, int out_dtype, void* stream);
+
 /* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd need for these sizes
  * (0 on invalid sizes).  The workspace is device memory, 256-byte aligned,
  * owned by the caller; its contents need not be initialised and are not
@@ -224,7 +246,8 @@ int qlora_device_status(void* stream);
 #define QLORA_KERNEL_GRAD_GEMM 6   /* dA^T = X^T V, dB = dY^T U (partials)    */
 #define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
 #define QLORA_KERNEL_FWD_DECODE 8  /* small-M forward (M <= 32, r <= 64)     */
-#define QLORA_KERNEL_COUNT 9
+#define QLORA_KERNEL_MERGE 9       /* adapter merge into the 16-bit base      */
+#define QLORA_KERNEL_COUNT 10
 int qlora_timing_enable(int on);
 /* Number of kernels the library has enqueued since it was loaded (all
  * devices, all streams), counted whether or not timing is enabled. */
