@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     qlora_nf4_codebook,
     qlora_quantize_nf4_dq,
     qlora_quantize_nf4,
+    qlora_selftest_device_timeout,
     qlora_strerror,
     qlora_timing_collect,
     qlora_timing_enable,

@@ -48,6 +48,7 @@ _SIGNATURES = {
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "qlora_selftest_device_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_timing_enable": (ctypes.c_int, [ctypes.c_int]),
     "qlora_timing_collect": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]),
     "qlora_launch_count": (ctypes.c_int64, []),
@@ -313,3 +314,10 @@ def qlora_timing_collect() -> dict:
 def qlora_launch_count() -> int:
     """Kernels the library has enqueued since it was loaded."""
     return int(load().qlora_launch_count())
+
+
+def qlora_selftest_device_timeout(waited_ns=None, stream=None):
+    """Enqueue the library's expired-wait diagnostic (see include/qlora_nf4.h)."""
+    if waited_ns is not None:
+        _dev(waited_ns, torch.int64, "waited_ns", (1,))
+    _check(load().qlora_selftest_device_timeout(_ptr(waited_ns), _stream(stream)), "qlora_selftest_device_timeout")

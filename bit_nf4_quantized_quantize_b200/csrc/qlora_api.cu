@@ -480,6 +480,26 @@ int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat,
   return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM);
 }
 
+// ------------------------------------------------------------------ failure-path self-test
+// One warp waits, bounded, on an mbarrier that nothing arrives at.  The wait
+// gives up after kWaitLimitNs, latches the device error flag (as any kernel's
+// expired wait does) and the kernel exits normally; *waited_ns (if given)
+// receives how long it waited.
+__global__ void selftest_wait_kernel(unsigned long long* waited_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const uint64_t t0 = globaltimer_ns();
+  const bool ok = mbar_wait(&bar, 0, &abort_word);
+  __syncwarp();
+  if (threadIdx.x == 0 && waited_ns != nullptr) *waited_ns = ok ? 0ull : globaltimer_ns() - t0;
+}
+
 // ------------------------------------------------------------------ fixed scratch
 // Scratch of qlora_linear_fwd_noalloc: a file-scope device array, so that the
 // library never allocates for that entry point.  Every GPU that loads the
@@ -846,6 +866,16 @@ int qlora_timing_collect(double* ms, int64_t* counts, int n_kinds) {
   }
   g_timing_recs.clear();
   return rc;
+}
+
+int qlora_selftest_device_timeout(unsigned long long* waited_ns, void* stream) {
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  selftest_wait_kernel<<<1, 32, 0, st>>>(waited_ns);
+  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return QLORA_OK;
 }
 
 int qlora_device_status(void* stream) {

@@ -220,6 +220,17 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Diagnostic for the failure path.  Enqueues one warp that waits, bounded, on
+ * an mbarrier nothing arrives at: the wait gives up after the library's limit
+ * (2 s of %globaltimer), latches the device error flag exactly as an expired
+ * wait in any kernel does, and the kernel exits normally (no trap, fault or
+ * hang; the context stays usable).  qlora_device_status then returns
+ * QLORA_ERR_DEVICE_TIMEOUT once.  waited_ns: device uint64 receiving the
+ * wait's duration in ns, or NULL.  The pages have no counterpart.
+ */
+int qlora_selftest_device_timeout(unsigned long long* waited_ns, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error flag of the
  * current device: QLORA_OK, QLORA_ERR_DEVICE_TIMEOUT if a kernel's bounded
  * wait expired since the last call, or QLORA_ERR_CUDA if the stream reports a
