@@ -13,7 +13,9 @@
 #include <cstdint>
 #include <cstring>
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 #include <vector>
 
@@ -389,22 +391,73 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms) {
   return w;
 }
 
-// Cluster size for the small-M split of the single-CTA fused kernel (one CTA
-// per SM): the most ranks (<= 8) that keep tiles x S within one wave and give
-// every rank at least two reduction steps.
-int pick_split(int tiles, int k_steps, int num_sms) {
+
+// How many clusters of S CTAs (along z) of `kern` can be resident at once,
+// from the occupancy API (it accounts for how clusters pack into the GPU's
+// processing clusters), cached per kernel, device and S.
+int cluster_capacity(const void* kern, int threads, size_t smem, int S, int dev) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int>, int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_tuple(kern, dev, S);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, static_cast<unsigned>(S));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 1;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = static_cast<unsigned>(S);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache.emplace(key, n);
+  return n;
+}
+
+// The largest split S <= 8 of k_steps reduction steps over a cluster along z
+// such that every tile's cluster is resident at once (one wave) and every
+// rank gets at least min_per steps; 1 when no split fits.  pow2: S must be a
+// power of two (the kernel's reduction divides 128 tile rows by S).
+int one_wave_split(const void* kern, int threads, size_t smem, int tiles, int k_steps, int min_per, bool pow2,
+                   int dev) {
   int S = 1;
-  while (S < 8 && tiles * (S + 1) <= num_sms && (S + 1) * 2 <= k_steps) ++S;
+  for (int c = 2; c <= 8; ++c) {
+    if (pow2 && (c & (c - 1)) != 0) continue;
+    const int per = (k_steps + c - 1) / c;
+    if (per < min_per || (c - 1) * per >= k_steps) continue;   // every rank gets work
+    if (tiles <= cluster_capacity(kern, threads, smem, c, dev)) S = c;
+  }
   return S;
 }
 
-// Cluster size for a split-K adapter product: the largest power of two <= 8
-// that keeps tiles x S within one wave of 2 CTAs per SM and gives every rank
-// at least one reduction step.
-int pick_cluster(int tiles, int k_steps, int num_sms) {
+// Split of a split-K adapter product (qlora_lora_kernel): the largest power
+// of two <= 8 with tiles x S <= 2 x SMs and at least one reduction step per
+// rank.  (The occupancy API reports one CTA of this kernel per SM; splits
+// sized to that measured slower on the train4096 shapes: dA/dB 26.7 us at
+// S = 2 against 23.9 us at S = 4.)
+int lora_cluster(int tiles, int k_steps, int num_sms) {
   int S = 1;
   while (S < 8 && tiles * S * 2 <= 2 * num_sms && S * 2 <= k_steps) S *= 2;
   return S;
+}
+
+// Split of the small-M single-CTA fused kernel (one CTA per 128 x 256 tile):
+// at least two reduction steps per rank.
+template <int BSRC>
+int gemm_split(int tiles, int k_steps, int dev) {
+  using L = GemmSmem<256, 4, BSRC, 8, 1>;
+  return one_wave_split(reinterpret_cast<const void*>(qlora_gemm_kernel<256, 4, false, BSRC, kOutBf16, 8, 1>),
+                        64 + 32 * 8, L::kDynBytes, tiles, k_steps, 2, false, dev);
 }
 
 template <bool A_MN, bool B_MN>
@@ -470,7 +523,7 @@ int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat,
   if (!map_bf16(&ta, X, M, K, 64, 128) || !map_bf16(&tb, Amat, r, K, 64, 64)) return QLORA_ERR_CUDA;
   const int k_steps = static_cast<int>(K / 64);
   const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
-  const int S = pick_cluster(tiles, k_steps, num_sms);
+  const int S = lora_cluster(tiles, k_steps, num_sms);
   LoraArgs la{};
   la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, plain, scaled, 0);
   la.p[1] = la.p[0];
@@ -701,7 +754,7 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     return QLORA_ERR_CUDA;
   // small M: split the reduction over a cluster of up to 8 CTAs (DSMEM sum)
   const int tiles = static_cast<int>((M + 127) / 128) * static_cast<int>((n_out + 255) / 256);
-  const int S = pick_split(tiles, g.k_steps, sms);
+  const int S = gemm_split<kBDeqK>(tiles, g.k_steps, dev);
   g.steps_per_split = (g.k_steps + S - 1) / S;
   const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((n_out + 255) / 256),
                   static_cast<unsigned>(S));
@@ -756,7 +809,7 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     if (!map_bf16(&ta, dY, M, N, 64, 128) || !map_bf16(&tb, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
     const int k_steps = N / 64;
     const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
-    const int S = pick_cluster(tiles, k_steps, sms);
+    const int S = lora_cluster(tiles, k_steps, sms);
     LoraArgs la{};
     la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, V, Vs, 0);
     la.p[1] = la.p[0];
@@ -804,7 +857,7 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
           !map_bf16(&ta2, Vs, M, r, 64, 128) || !map_bf16(&tb2, A, r, K, 64, 64))
         return QLORA_ERR_CUDA;
       const int tiles = static_cast<int>((M + 127) / 128) * ((K + 255) / 256);
-      const int S = pick_split(tiles, g.k_steps, sms);
+      const int S = gemm_split<kBDeqMN>(tiles, g.k_steps, dev);
       g.steps_per_split = (g.k_steps + S - 1) / S;
       const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256),
                       static_cast<unsigned>(S));
@@ -821,7 +874,7 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     const int k_steps = static_cast<int>((M + 63) / 64);
     const int tiles_a = ((K + 127) / 128) * (rpad / 64);
     const int tiles_b = ((N + 127) / 128) * (rpad / 64);
-    const int S = pick_cluster(tiles_a + tiles_b, k_steps, sms);
+    const int S = lora_cluster(tiles_a + tiles_b, k_steps, sms);
     LoraArgs la{};
     la.p[0] = lora_problem(K, k_steps, S, rpad, kLoraOutTransposed, dA, nullptr, K);
     la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0);
