@@ -68,6 +68,11 @@ def _load():
             lib.oracle_quantize_nf4.restype = ctypes.c_int
             lib.oracle_quantize_nf4.argtypes = [P, i64, P, P, P]
             lib.oracle_double_quant.argtypes = [P, i64, P, P]
+            lib.oracle_double_quant_fp8.argtypes = [P, i64, P, P]
+            lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+            lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_to_f32.restype = ctypes.c_float
+            lib.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
             lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
             lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.oracle_dequant.argtypes = [P, P, P, i64, P, P, P]
@@ -132,6 +137,35 @@ def double_quant(absmax: np.ndarray):
     s2 = np.zeros((nb + GROUP - 1) // GROUP, np.float32)
     _load().oracle_double_quant(_p(a), nb, _p(q8), _p(s2))
     return q8, s2
+
+
+def double_quant_fp8(absmax: np.ndarray):
+    """FP8-E4M3 re-quantization of absmax in groups of 256 -> (q8 u8[nb], s2 f32 with the sign bit set)."""
+    a = np.ascontiguousarray(absmax, np.float32).reshape(-1)
+    nb = a.size
+    q8 = np.zeros(nb, np.uint8)
+    s2 = np.zeros((nb + GROUP - 1) // GROUP, np.float32)
+    _load().oracle_double_quant_fp8(_p(a), nb, _p(q8), _p(s2))
+    return q8, s2
+
+
+def f32_to_e4m3(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, np.float32).reshape(-1)
+    f = _load().oracle_f32_to_e4m3
+    return np.array([f(float(v)) for v in x], np.uint8)
+
+
+def e4m3_to_f32(b) -> np.ndarray:
+    b = np.ascontiguousarray(b, np.uint8).reshape(-1)
+    f = _load().oracle_e4m3_to_f32
+    return np.array([f(int(v)) for v in b], np.float32)
+
+
+def quantize_nf4_dq_fp8(w: np.ndarray, table32: np.ndarray | None = None):
+    """Two-level quantization with the FP8 second stage -> (codes, q8, s2, absmax)."""
+    codes, absmax = quantize_nf4(w, table32)
+    q8, s2 = double_quant_fp8(absmax)
+    return codes, q8, s2, absmax
 
 
 def quantize_nf4_dq(w: np.ndarray, table32: np.ndarray | None = None):

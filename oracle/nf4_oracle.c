@@ -31,6 +31,9 @@
  *     q = min(255, round-half-even(fp32(absmax/s2))), s2 == 0 gives q = 0;
  *   - dequant: w = bf16( fp32( c[code] * fp32(q * s2) ) );
  *   - single quantization (second stage off): w = bf16( fp32( c[code] * absmax ) );
+ *   - FP8 reading of the second stage ("8bit量子化（FP8相当）"): s2 = fp32(c2/448),
+ *     q = E4M3(fp32(absmax/s2)) rounded to nearest even and saturated at 448,
+ *     stored with the sign bit of s2 set to mark the group's format;
  *   - adapter merge: into the 16-bit base, not the 4-bit one (p4), as one
  *     rounding of the fp64 value bf16(W) + s * sum_j B[n,j] A[j,k].
  *
@@ -196,6 +199,57 @@ void oracle_double_quant(const float* absmax, int64_t nb, uint8_t* q8, float* s2
     }
 }
 
+/* FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no   */
+/* infinities, largest finite value 448, smallest subnormal 2^-9).  Encode:  */
+/* round to nearest even, then clamp to 448 (saturating); input >= 0.        */
+uint8_t oracle_f32_to_e4m3(float x) {
+    if (!(x > 0.0f)) return 0;
+    double a = (double)x;
+    int e;
+    frexp(a, &e);                        /* a = m * 2^e, 0.5 <= m < 1          */
+    int ue = e - 4;                      /* 4 significant bits                 */
+    if (ue < -9) ue = -9;                /* subnormal step 2^-9                */
+    double r = ldexp(rint(ldexp(a, -ue)), ue);
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return 0;
+    int E;
+    double m = frexp(r, &E);
+    int ef = E - 1 + 7;                  /* biased exponent of r               */
+    if (ef <= 0) return (uint8_t)ldexp(r, 9);          /* subnormal: r / 2^-9 */
+    return (uint8_t)((ef << 3) | ((int)ldexp(m, 4) - 8));
+}
+
+float oracle_e4m3_to_f32(uint8_t b) {
+    int e = (b >> 3) & 15, m = b & 7;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (float)((b & 0x80) ? -v : v);
+}
+
+/* The FP8 reading of the second stage of p1 §5-2 ("8bit量子化（FP8相当）"),     */
+/* [p2] "Double Quantization の仕組み" (c1 quantized to 8 bits with the FP32  */
+/* c2 above it): per group of 256 blocks, s = fp32(c2 / 448) so that the    */
+/* group maximum maps to E4M3's largest finite value, q = E4M3(fp32(absmax  */
+/* / s)), q = 0 when s == 0.  s2 stores -s: its sign bit marks the group as */
+/* FP8 (every linear-format s2 is >= 0), and c1' = fp32(E4M3 value * |s2|). */
+void oracle_double_quant_fp8(const float* absmax, int64_t nb, uint8_t* q8, float* s2) {
+    int64_t ng = (nb + ORACLE_GROUP - 1) / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t g = 0; g < ng; ++g) {
+        int64_t b0 = g * ORACLE_GROUP;
+        int64_t b1 = b0 + ORACLE_GROUP < nb ? b0 + ORACLE_GROUP : nb;
+        float c2 = 0.0f;
+        for (int64_t b = b0; b < b1; ++b) if (absmax[b] > c2) c2 = absmax[b];
+        volatile float s = c2 / 448.0f;
+        s2[g] = -s;
+        for (int64_t b = b0; b < b1; ++b) {
+            if (s == 0.0f) { q8[b] = 0; continue; }
+            volatile float ratio = absmax[b] / s;
+            q8[b] = oracle_f32_to_e4m3(ratio);
+        }
+    }
+}
+
+
 /* Round an fp32 value to bf16 (round to nearest, ties to even), returned as */
 /* its 16-bit pattern.  NaN stays a quiet NaN.                               */
 uint16_t oracle_f32_to_bf16(float f) {
@@ -223,7 +277,8 @@ void oracle_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2,
     for (int64_t i = 0; i < n; ++i) {
         int64_t b = i / ORACLE_BLOCK, g = b / ORACLE_GROUP;
         int code = (i & 1) ? (codes[i / 2] >> 4) : (codes[i / 2] & 15);
-        volatile float c1 = (float)q8[b] * s2[g];
+        /* a set sign bit marks an FP8-format group (oracle_double_quant_fp8) */
+        volatile float c1 = signbit(s2[g]) ? oracle_e4m3_to_f32(q8[b]) * -s2[g] : (float)q8[b] * s2[g];
         volatile float w32 = table[code] * c1;
         if (out_f32) out_f32[i] = w32;
         if (out_bf16) out_bf16[i] = oracle_f32_to_bf16(w32);

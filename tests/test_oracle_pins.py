@@ -246,6 +246,67 @@ def test_double_quant_zero_and_subnormal_groups():
     assert s2[0] == 0 and np.all(q8 == 0)
 
 
+# --------------------------------------------------- FP8 reading of the DQ
+def _torch_e4m3_bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_every_code_matches_torch():
+    codes = np.array([b for b in range(256) if b not in (0x7F, 0xFF)], np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(oracle.e4m3_to_f32(codes).view(np.uint32), ref.view(np.uint32))
+
+
+def test_e4m3_encode_is_round_to_nearest_even_and_saturates():
+    g = np.random.default_rng(31)
+    x = np.concatenate([g.uniform(0, 448, 3000), 2.0 ** g.uniform(-12, 8.8, 3000)]).astype(np.float32)
+    # exact midpoints between neighbouring E4M3 values (ties go to the even mantissa)
+    vals = oracle.e4m3_to_f32(np.arange(0, 0x7E, dtype=np.uint8)).astype(np.float64)
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, vals.astype(np.float32)])
+    x = x[x <= 448]
+    assert np.array_equal(oracle.f32_to_e4m3(x), _torch_e4m3_bits(x))
+    # above the largest finite value the conversion saturates to 448 (code 0x7E)
+    assert np.all(oracle.f32_to_e4m3(np.array([448.5, 463.9, 464.0, 470.0, 1e30], np.float32)) == 0x7E)
+
+
+def test_double_quant_fp8_cases_and_error_bound():
+    # a group of equal constants: every q is 448's code and fp32(448 * |s2|) is within 1 ulp of c2
+    a = np.full(256, 0.37, np.float32)
+    q8, s2 = oracle.double_quant_fp8(a)
+    assert np.all(q8 == 0x7E) and np.signbit(s2[0])
+    assert abs(np.float32(448) * -s2[0] - np.float32(0.37)) <= np.spacing(np.float32(0.37))
+    # zero group: q = 0, s2 = -0.0, dequant 0
+    q8, s2 = oracle.double_quant_fp8(np.zeros(300, np.float32))
+    assert np.all(q8 == 0) and np.all(s2 == 0) and np.all(np.signbit(s2))
+    # random constants: relative error <= 2^-4 in E4M3's normal range, <= 2^-10 |s2| below it
+    g = np.random.default_rng(32)
+    a = (2.0 ** g.uniform(-20, 0, 256 * 40)).astype(np.float32)
+    q8, s2 = oracle.double_quant_fp8(a)
+    s = np.repeat(-s2, 256)[: a.size].astype(np.float64)
+    c1 = (oracle.e4m3_to_f32(q8).astype(np.float32) * s.astype(np.float32)).astype(np.float64)
+    ratio = a / s
+    err = np.abs(c1 - a)
+    normal = ratio >= 2.0 ** -6
+    assert np.all(err[normal] <= a[normal] * 2.0 ** -4 * (1 + 1e-6))
+    assert np.all(err[~normal] <= s[~normal] * 2.0 ** -10 * (1 + 1e-6))
+
+
+def test_dequant_fp8_matches_formula_in_numpy():
+    w = synth.weight(2, 0, 512, 512).reshape(-1)
+    codes, absmax = oracle.quantize_nf4(w)
+    q8, s2 = oracle.double_quant_fp8(absmax)
+    _, t32 = oracle.nf4_codebook()
+    w32, wb = oracle.dequant(codes, q8, s2, w.size)
+    un = np.stack([codes & 15, codes >> 4], 1).reshape(-1)
+    qv = torch.from_numpy(q8.copy()).view(torch.float8_e4m3fn).float().numpy()
+    c1 = (qv * np.repeat(-s2, 256)[: q8.size]).astype(np.float32)
+    ref = (t32[un] * np.repeat(c1, 64)).astype(np.float32)
+    assert np.array_equal(w32.view(np.uint32), ref.view(np.uint32))
+    # the 8-bit codes cost the same 4.127 bit/param as the linear format
+    assert 8 * (codes.nbytes + q8.nbytes + s2.nbytes) / w.size == 4 + 8 / 64 + 32 / (64 * 256)
+
+
 # ---------------------------------------------------------------- overhead
 def test_overheads_match_the_pages_closed_forms():
     G = GOLDEN
