@@ -389,22 +389,32 @@ def run_quantize_stream(q, dev, peaks, seed=5, reps=3):
             "algorithmic_bytes": byts, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "passes": reps}
 
 
-def run_single_quant(q, dev, peaks, reps=20):
-    """The train4096 layer with the second quantization stage off: quantize GB/s
-    (4 B read, 0.5 + 4/64 B written per weight) and fwd+bwd TFLOP/s."""
+def run_quant_variant(q, dev, peaks, variant, reps=20):
+    """The train4096 layer with another form of the second quantization stage
+    ("single": off, 4 B read and 0.5 + 4/64 B written per weight; "fp8": the
+    FP8-E4M3 reading, the same bytes as the linear form): quantize GB/s and
+    fwd+bwd TFLOP/s."""
     import torch
     N, K, M, r, alpha = N_OUT, K_IN, M_TOK, RANK, ALPHA
     gen = torch.Generator(device=dev)
     gen.manual_seed(3)
     W = gpu_weight(gen, N, K, "normal", dev)
     codes = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
-    absmax = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    qbytes = 4 * N * K + N * K // 2 + 4 * (N * K // 64)
+    if variant == "single":
+        q8 = None
+        s2 = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
+        qbytes = 4 * N * K + N * K // 2 + 4 * (N * K // 64)
+        qfn = lambda: q.qlora_quantize_nf4(W, codes, s2)
+    else:
+        q8 = torch.empty(N * K // 64, dtype=torch.uint8, device=dev)
+        s2 = torch.empty((N * K // 64 + 255) // 256, dtype=torch.float32, device=dev)
+        qbytes = quant_bytes(N, K)
+        qfn = lambda: q.qlora_quantize_nf4_dq_fp8(W, codes, q8, s2)
 
     def quant():
         flush.fill_(0.0)
-        q.qlora_quantize_nf4(W, codes, absmax)
+        qfn()
 
     # time the quantize launches alone: events around each, after an L2 flush
     for _ in range(3):
@@ -414,7 +424,7 @@ def run_single_quant(q, dev, peaks, reps=20):
         flush.fill_(0.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        q.qlora_quantize_nf4(W, codes, absmax)
+        qfn()
         e1.record()
         ev.append((e0, e1))
     torch.cuda.synchronize()
@@ -431,17 +441,19 @@ def run_single_quant(q, dev, peaks, reps=20):
     ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
 
     def step():
-        q.qlora_linear_fwd(codes, None, absmax, N, K, L["X"], L["A"], L["B"], alpha, Y=Y, U_save=U, workspace=ws)
-        q.qlora_linear_bwd(codes, None, absmax, N, K, L["X"], L["A"], L["B"], alpha, L["dY"], U_saved=U, dX=dX,
+        q.qlora_linear_fwd(codes, q8, s2, N, K, L["X"], L["A"], L["B"], alpha, Y=Y, U_save=U, workspace=ws)
+        q.qlora_linear_bwd(codes, q8, s2, N, K, L["X"], L["A"], L["B"], alpha, L["dY"], U_saved=U, dX=dX,
                            dA=dA, dB=dB, workspace=ws)
 
     ms = time_region(step, 3, 10)
     rc = q.qlora_device_status()
     if rc != 0:
-        raise RuntimeError(f"device status after the single-quantization region: {q.qlora_strerror(rc)}")
+        raise RuntimeError(f"device status after the {variant} quantization region: {q.qlora_strerror(rc)}")
     tf = step_flops(M, N, K, r) / (ms * 1e-3) / 1e12
     gbs = qbytes / (q_ms * 1e-3) / 1e9
-    return {"workload": "train4096 layer, second quantization stage off (4.5 bit/param)",
+    what = "second quantization stage off (4.5 bit/param)" if variant == "single" else \
+        "FP8-E4M3 second quantization stage (4.127 bit/param)"
+    return {"workload": f"train4096 layer, {what}",
             "quantize_gbs": gbs, "quantize_frac": gbs / peaks["hbm_gbs"], "quantize_algorithmic_bytes": qbytes,
             "fwd_bwd_tflops": tf, "fwd_bwd_ms": ms}
 
@@ -481,7 +493,9 @@ def run_configs(q, dev, peaks):
     torch.cuda.empty_cache()
     out["llama65b_quantize_stream"] = run_quantize_stream(q, dev, peaks)
     torch.cuda.empty_cache()
-    out["train4096_single_quant"] = run_single_quant(q, dev, peaks)
+    out["train4096_single_quant"] = run_quant_variant(q, dev, peaks, "single")
+    torch.cuda.empty_cache()
+    out["train4096_fp8_dq"] = run_quant_variant(q, dev, peaks, "fp8")
     torch.cuda.empty_cache()
     out["train4096_merge_requantize"] = run_merge(q, dev, peaks)
     torch.cuda.empty_cache()

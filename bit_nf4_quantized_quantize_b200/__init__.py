@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     qlora_merge_adapter,
     qlora_nf4_codebook,
     qlora_quantize_nf4_dq,
+    qlora_quantize_nf4_dq_fp8,
     qlora_quantize_nf4,
     qlora_selftest_device_timeout,
     qlora_strerror,

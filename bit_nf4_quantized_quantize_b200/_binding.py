@@ -26,6 +26,8 @@ _SIGNATURES = {
     "qlora_nf4_codebook": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_quantize_nf4_dq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_quantize_nf4_dq_fp8": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_quantize_nf4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_merge_adapter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
@@ -150,6 +152,23 @@ def qlora_quantize_nf4_dq(W, codes=None, q8=None, s2=None, stream=None):
     s2 = torch.empty(ng, dtype=torch.float32, device=dev) if s2 is None else _dev(s2, torch.float32, "s2", (ng,))
     _check(load().qlora_quantize_nf4_dq(_ptr(W), N, K, _ptr(codes), _ptr(q8), _ptr(s2), _stream(stream)),
            "qlora_quantize_nf4_dq")
+    return codes, q8, s2
+
+
+def qlora_quantize_nf4_dq_fp8(W, codes=None, q8=None, s2=None, stream=None):
+    """NF4 + double quantization with the FP8-E4M3 second stage -> (codes, q8, s2);
+    s2 carries its sign bit set, which every consumer reads as the FP8 format."""
+    _dev(W, torch.float32, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [n_out, k_in]")
+    N, K = W.shape
+    nc, nb, ng = quant_sizes(N, K)
+    dev = W.device
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev) if codes is None else _dev(codes, torch.uint8, "codes", (nc,))
+    q8 = torch.empty(nb, dtype=torch.uint8, device=dev) if q8 is None else _dev(q8, torch.uint8, "q8", (nb,))
+    s2 = torch.empty(ng, dtype=torch.float32, device=dev) if s2 is None else _dev(s2, torch.float32, "s2", (ng,))
+    _check(load().qlora_quantize_nf4_dq_fp8(_ptr(W), N, K, _ptr(codes), _ptr(q8), _ptr(s2), _stream(stream)),
+           "qlora_quantize_nf4_dq_fp8")
     return codes, q8, s2
 
 

@@ -292,8 +292,7 @@ qlora_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     auto load_scale = [&](int ks) -> float {
       if (is_adapter || w_row >= args.n_cols) return 0.f;
       const int64_t blk = static_cast<int64_t>(w_row) * kblocks + ks;
-      if (args.q8 == nullptr) return __ldg(args.s2 + blk);   // single quantization: fp32 absmax
-      return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
+      return block_scale(args.q8, args.s2, blk);
     };
     // this warpgroup's steps are t = wg, wg + kDecWG, ...: scales two of them ahead
     float c1_a = (wg < n_steps) ? load_scale(step_begin + wg) : 0.f;

@@ -258,8 +258,7 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       else { wr = ks * 64 + (item & 63); kb = cb / 64 + (item >> 6); }
       if (wr >= args.w_rows || kb >= args.w_kblocks) return 0.f;
       const int64_t blk = static_cast<int64_t>(wr) * args.w_kblocks + kb;
-      if (args.q8 == nullptr) return __ldg(args.s2 + blk);   // single quantization: fp32 absmax
-      return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
+      return block_scale(args.q8, args.s2, blk);
     };
     // this warpgroup's main steps are ks = first, first+2, ...; prefetch two ahead
     const int first = (n_lora + wg) & 1;   // smallest ks with (n_lora + ks) % 2 == wg

@@ -316,8 +316,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int kb = (BSRC == kBDeqK) ? ks : kb_base;
         if (wr >= args.w_rows || kb >= args.w_kblocks) return 0.f;
         const int64_t blk = static_cast<int64_t>(wr) * args.w_kblocks + kb;
-        if (args.q8 == nullptr) return __ldg(args.s2 + blk);   // single quantization: fp32 absmax
-        return __fmul_rn(static_cast<float>(__ldg(args.q8 + blk)), __ldg(args.s2 + (blk >> 8)));
+        return block_scale(args.q8, args.s2, blk);
       };
       // scales are prefetched two steps ahead (c1_a: this step, c1_b: next)
       float c1_a = (n_main > 0) ? load_scale(step_begin) : 0.f;

@@ -85,6 +85,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ---------------------------------------------------------------- block scales
+// FP8 E4M3 (bias 7, 3 mantissa bits, no infinities) -> fp32, exact.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  const float v = e != 0u ? __uint_as_float(((e + 120u) << 23) | (m << 20))
+                          : __fmul_rn(static_cast<float>(m), 0.001953125f);   // m * 2^-9
+  return (b & 0x80u) ? -v : v;
+}
+
+// The combined scale c1 of 64-block `blk` of an NF4 weight, in its stored form:
+//   q8 == nullptr (single quantization): s2 holds the fp32 absmax of each block;
+//   linear 8-bit second stage:           c1 = fp32(q8 * s2[group]);
+//   FP8-E4M3 second stage (the group's s2 has its sign bit set):
+//                                        c1 = fp32(E4M3(q8) * |s2[group]|).
+__device__ __forceinline__ float block_scale(const uint8_t* q8, const float* s2, int64_t blk) {
+  if (q8 == nullptr) return __ldg(s2 + blk);
+  const uint32_t q = __ldg(q8 + blk);
+  const float sv = __ldg(s2 + (blk >> 8));
+  if (signbit(sv)) return __fmul_rn(e4m3_to_f32(q), -sv);
+  return __fmul_rn(static_cast<float>(q), sv);
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

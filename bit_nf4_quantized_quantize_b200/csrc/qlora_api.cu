@@ -620,8 +620,26 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_nf4_kernel<true>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
+    return launch_ex(quantize_nf4_kernel<kQuantLinear8>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
                      1, W, n_blocks, codes, q8, s2, tables());
+  });
+}
+
+int qlora_quantize_nf4_dq_fp8(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, uint8_t* q8, float* s2,
+                              void* stream) {
+  if (!W || !codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
+  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(s2) & 3u))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  const int64_t n_blocks = n_out * k_in / kBlock;
+  const int64_t groups = (n_blocks + kGroup - 1) / kGroup;
+  if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
+    return launch_ex(quantize_nf4_kernel<kQuantFp8>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st,
+                     1, 1, W, n_blocks, codes, q8, s2, tables());
   });
 }
 
@@ -638,7 +656,7 @@ int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* cod
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* no_q8 = nullptr;
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_nf4_kernel<false>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
+    return launch_ex(quantize_nf4_kernel<kQuantSingle>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
                      1, W, n_blocks, codes, no_q8, absmax, tables());
   });
 }

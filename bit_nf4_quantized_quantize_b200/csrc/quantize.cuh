@@ -5,14 +5,14 @@
 // absmax constants in groups of 256, one fp32 second-level constant; without
 // that second stage the fp32 absmax constants are stored as they are).
 //
-// quantize_nf4_kernel<kDQ>: one CTA of 512 threads per group of 256 blocks (16384
+// quantize_nf4_kernel<kMode>: one CTA of 512 threads per group of 256 blocks (16384
 // weights, 64 KiB of fp32 input).  Eight threads share a 64-block (8
 // consecutive weights each, two 16-byte loads), so a warp reads 1 KiB
 // contiguous per pass; the block absmax is a 3-step xor-shuffle max.  The
 // group's 256 absmax values then stay in shared memory for the second-level
 // quantization, so the fp32 constants never go to HBM.  Traffic per weight:
-// 4 B read, 0.5 + 1/64 + 4/16384 B written (kDQ), or 0.5 + 4/64 B written
-// when the second stage is off and the absmax constants are stored.
+// 4 B read, 0.5 + 1/64 + 4/16384 B written with a second stage, or 0.5 + 4/64
+// B written when the second stage is off and the absmax constants are stored.
 //
 // Nearest level.  The code of n = fp32(w / absmax) is #{i : n >= thr_i}, thr_i
 // the smallest fp32 above the exact midpoint of levels i and i+1.  Cells of
@@ -50,9 +50,13 @@ struct Nf4Tables {
 
 constexpr int kQuantThreads = 512;  // 16 warps; 8 threads per 64-block, 4 passes of 64 blocks
 
-// kDQ: q8 / s2 receive the second-level quantization of the absmax constants.
-// !kDQ: q8 is unused and s2 receives the n_blocks fp32 absmax constants.
-template <bool kDQ>
+// Second stage of the quantizer.
+enum QuantMode : int {
+  kQuantSingle = 0,   // none: s2 receives the n_blocks fp32 absmax constants, q8 unused
+  kQuantLinear8 = 1,  // q8 = min(255, rint(fp32(absmax / s2))), s2 = fp32(c2 / 255)
+  kQuantFp8 = 2,      // q8 = E4M3(fp32(absmax / s)), s = fp32(c2 / 448), stored as s2 = -s
+};
+template <int kMode>
 __global__ void __launch_bounds__(kQuantThreads, 2)
 quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
                     uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
@@ -134,13 +138,13 @@ quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __re
       }
       *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
       if (sub == 0) {
-        if (kDQ) s_absmax[lb] = am;
+        if (kMode != kQuantSingle) s_absmax[lb] = am;
         else s2[b_first + lb] = am;
       }
     }
   }
   griddep_launch_dependents();
-  if (!kDQ) return;
+  if (kMode == kQuantSingle) return;
   __syncthreads();
 
   // Second level: c2 = max of the group's absmax, s2 = fp32(c2/255),
@@ -158,23 +162,29 @@ quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __re
     float c2 = s_warpmax[0];
 #pragma unroll
     for (int w = 1; w < kGroup / 32; ++w) c2 = fmaxf(c2, s_warpmax[w]);
-    const float sc = __fdiv_rn(c2, 255.f);
+    const float sc = __fdiv_rn(c2, kMode == kQuantFp8 ? 448.f : 255.f);
     if (tid < nb) {
-      int q = 0;
+      uint32_t q = 0;
       if (sc != 0.f) {
         const float ratio = __fdiv_rn(s_absmax[tid], sc);
-        q = min(255, __float2int_rn(ratio));  // round half to even
+        if (kMode == kQuantFp8) {
+          uint16_t pr;   // round to nearest even, saturating at 448; both halves hold the same code
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(ratio), "f"(ratio));
+          q = pr & 0xFFu;
+        } else {
+          q = static_cast<uint32_t>(min(255, __float2int_rn(ratio)));  // round half to even
+        }
       }
       q8[b_first + tid] = static_cast<uint8_t>(q);
     }
-    if (tid == 0) s2[g] = sc;
+    // the FP8 form stores -s: the sign bit marks the group's format
+    if (tid == 0) s2[g] = kMode == kQuantFp8 ? -sc : sc;
   }
 }
 
-// Dense dequantization: w = fp32(level[code] * fp32(q * s2)), fp32 or bf16 out;
-// with q8 == nullptr (single quantization) s2 holds the fp32 absmax per block
-// and w = fp32(level[code] * absmax).  One thread per 8 consecutive weights
-// (4 packed bytes).
+// Dense dequantization: w = fp32(level[code] * c1), c1 the block scale in any
+// of its stored forms (block_scale), fp32 or bf16 out.  One thread per 8
+// consecutive weights (4 packed bytes).
 template <bool kBf16>
 __global__ void __launch_bounds__(256)
 dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8,
@@ -188,8 +198,7 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ q8
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(codes) + i);
     const int64_t blk = (i * 8) / kBlock;
-    const float c1 = q8 == nullptr ? __ldg(s2 + blk)
-                                   : __fmul_rn(static_cast<float>(__ldg(q8 + blk)), __ldg(s2 + blk / kGroup));
+    const float c1 = block_scale(q8, s2, blk);
     float w[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(s_level[(p >> (4 * j)) & 15u], c1);

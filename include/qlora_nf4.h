@@ -29,7 +29,10 @@
  *                                nibble of byte j;
  *     q8     uint8_t[N*K/64]     8-bit absmax constant of each 64-block;
  *     s2     float[ceil(N*K/16384)]  fp32 second-level constant of each group
- *                                of 256 consecutive blocks;
+ *                                of 256 consecutive blocks.  Its sign bit
+ *                                gives the group's 8-bit format: clear =
+ *                                linear (c1 = q8 * s2), set = FP8-E4M3
+ *                                (c1 = E4M3(q8) * |s2|);
  *   or, with single quantization (the second stage off, 4.5 bit/param), two:
  *     codes  as above;  q8 = NULL;
  *     s2     float[N*K/64]       the fp32 absmax constant of each 64-block.
@@ -95,6 +98,19 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in,
                           uint8_t* codes, uint8_t* q8, float* s2, void* stream);
 
 /*
+ * The same with the FP8 reading of the second stage ("QLoRAの理論と実装" §5-2:
+ * "8bit量子化（FP8相当）"): per group of 256 blocks s = fp32(c2 / 448), so the
+ * group maximum maps to E4M3's largest finite value, and
+ * q = E4M3(fp32(absmax / s)), rounded to nearest even and saturated at 448
+ * (q = 0 when s == 0).  s2 receives -s: the sign bit marks the FP8 format,
+ * and every call that reads (codes, q8, s2) decodes c1 = fp32(E4M3(q) * s).
+ * Same buffers and sizes as qlora_quantize_nf4_dq; codes are identical.
+ * One kernel launch.
+ */
+int qlora_quantize_nf4_dq_fp8(const float* W, int64_t n_out, int64_t k_in,
+                              uint8_t* codes, uint8_t* q8, float* s2, void* stream);
+
+/*
  * Blockwise NF4 quantization without the second stage (single quantization):
  * "QLoRAの理論と実装" §5-1 steps 1-2 alone; §5-2's memory arithmetic prices it
  * at 4 + 32/64 = 4.5 bit/param, and the page's bitsandbytes listing selects it
@@ -111,8 +127,9 @@ int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in,
 
 /*
  * Dequantization to a dense N x K matrix ("QLoRAの理論と実装" §5-1 step 3 with
- * the two-level constant):  w = fp32(level[code] * fp32(q8 * s2)), or with
- * q8 == NULL w = fp32(level[code] * absmax) (s2 = absmax), written as
+ * the two-level constant):  w = fp32(level[code] * c1) with c1 = fp32(q8 * s2)
+ * (or fp32(E4M3(q8) * |s2|) for an FP8 group), or with q8 == NULL
+ * w = fp32(level[code] * absmax) (s2 = absmax), written as
  * fp32 (out_dtype QLORA_OUT_FP32) or rounded to nearest-even bf16
  * (QLORA_OUT_BF16).  `out` is device memory of N*K elements.  This is for
  * tests and export; the linear layer never materialises it.

@@ -20,12 +20,14 @@ from common import REL_L2_TOL, bf16_to_np_f64, bits_f64, oracle_weight, oracle_w
 pytestmark = pytest.mark.gpu
 
 
-def run_case(inp, rows=None, check_bwd=True, dy_rows=None, single=False):
+def run_case(inp, rows=None, check_bwd=True, dy_rows=None, single=False, fp8=False):
     N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
     Wd = torch.from_numpy(inp["W"]).cuda()
     if single:
         codes, s2 = q.qlora_quantize_nf4(Wd)   # second stage off: s2 = fp32 absmax
         q8 = None
+    elif fp8:
+        codes, q8, s2 = q.qlora_quantize_nf4_dq_fp8(Wd)
     else:
         codes, q8, s2 = q.qlora_quantize_nf4_dq(Wd)
     X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
@@ -37,7 +39,13 @@ def run_case(inp, rows=None, check_bwd=True, dy_rows=None, single=False):
         res.update(dX=dX, dA=dA, dB=dB)
     assert q.qlora_device_status() == 0
     # oracle on the same inputs
-    What = oracle_weight_single(inp["W"])[2] if single else oracle_weight(inp["W"])[3]
+    if single:
+        What = oracle_weight_single(inp["W"])[2]
+    elif fp8:
+        rc, rq, rs, _ = oracle.quantize_nf4_dq_fp8(inp["W"].reshape(-1))
+        What = bits_f64(oracle.dequant(rc, rq, rs, N * K)[1]).reshape(N, K)
+    else:
+        What = oracle_weight(inp["W"])[3]
     Xo, Ao, Bo, dYo = (bits_f64(inp[k]) for k in ("X", "A", "B", "dY"))
     Yr, Ur = oracle.linear_fwd(Xo, What, Ao, Bo, alpha, rows=rows)
     sel = slice(None) if rows is None else rows
@@ -150,3 +158,14 @@ def test_single_quantization_linear(M, N, K, r):
     """The layer on a weight without the second quantization stage (q8 = NULL,
     s2 = fp32 absmax per block): forward and backward against the oracle."""
     run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=700 + M), single=True)
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (1, 4096, 4096, 8),      # few-token path
+    (40, 512, 768, 8),       # tiled path
+    (300, 512, 768, 64),     # CTA-pair path
+])
+def test_fp8_second_stage_linear(M, N, K, r):
+    """The layer on a weight whose second stage is FP8-E4M3 (sign-tagged s2):
+    forward and backward against the oracle."""
+    run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=800 + M), fp8=True)

@@ -70,6 +70,26 @@ def check_exact_single(W: np.ndarray, dequant=True):
         assert np.array_equal(db.reshape(-1).view(np.uint16), wb)
 
 
+def check_exact_fp8(W: np.ndarray, dequant=True):
+    """FP8 second stage: codes, q8 and s2 (sign bit included) bit-exact; codes
+    identical to the linear form's; dense dequant bit-exact."""
+    N, K = W.shape
+    Wd = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    codes, q8, s2 = q.qlora_quantize_nf4_dq_fp8(Wd)
+    codes_lin, _, _ = q.qlora_quantize_nf4_dq(Wd)
+    rc, rq, rs, _ = oracle.quantize_nf4_dq_fp8(W.reshape(-1))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(q8.cpu().numpy(), rq)
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert torch.equal(codes, codes_lin)
+    if dequant:
+        w32, wb = oracle.dequant(rc, rq, rs, N * K)
+        d32 = q.qlora_dequant(codes, q8, s2, N, K, dtype=torch.float32).cpu().numpy().reshape(-1)
+        db = q.qlora_dequant(codes, q8, s2, N, K, dtype=torch.bfloat16).view(torch.int16).cpu().numpy()
+        assert np.array_equal(d32.view(np.uint32), w32.view(np.uint32))
+        assert np.array_equal(db.reshape(-1).view(np.uint16), wb)
+
+
 def edge_case_weight():
     _, t32 = oracle.nf4_codebook()
     blocks = []
@@ -109,6 +129,14 @@ def edge_case_weight():
 
 def test_edge_case_blocks_exact():
     check_exact(edge_case_weight())
+
+
+def test_fp8_second_stage_exact():
+    check_exact_fp8(synth.weight(1, 0, 256, 256))
+    check_exact_fp8(synth.weight(11, 0, 3, 6400))              # ragged last group
+    check_exact_fp8(edge_case_weight())                          # zero, subnormal, huge blocks
+    check_exact_fp8(synth.weight(3, 0, 4096, 4096))
+    check_exact_fp8(synth.weight(5, 0, 512, 8192, "student_t4"))  # wide spread of absmax within groups
 
 
 def test_single_quant_exact():
