@@ -69,6 +69,8 @@ def _load():
             lib.oracle_quantize_nf4.argtypes = [P, i64, P, P, P]
             lib.oracle_double_quant.argtypes = [P, i64, P, P]
             lib.oracle_double_quant_fp8.argtypes = [P, i64, P, P]
+            lib.oracle_philox4x32_10.argtypes = [P, P, P]
+            lib.oracle_dropout_keep.argtypes = [i64, i64, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_uint64, P]
             lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
             lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
             lib.oracle_e4m3_to_f32.restype = ctypes.c_float
@@ -221,6 +223,57 @@ def merge_adapter(W: np.ndarray, A_bits: np.ndarray, B_bits: np.ndarray, alpha: 
     out = np.zeros((N, K), np.uint16)
     _load().oracle_merge_adapter(_p(W), N, K, _p(A_bits), _p(B_bits), r, float(alpha), _p(out))
     return out
+
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """One Philox4x32-10 block: 4 uint32 outputs for a 4-word counter and 2-word key."""
+    c = np.ascontiguousarray(ctr, np.uint32)
+    k = np.ascontiguousarray(key, np.uint32)
+    out = np.zeros(4, np.uint32)
+    _load().oracle_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def dropout_threshold(p: float) -> int:
+    """Integer keep threshold floor(p * 2^32) (clamped to 2^32 - 1); element kept iff its word >= it."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("dropout probability must be in [0, 1)")
+    return min(int(np.floor(p * 4294967296.0)), 0xFFFFFFFF)
+
+
+def dropout_keep(M: int, K: int, p: float, seed: int, offset: int) -> np.ndarray:
+    """uint8 [M, K] keep mask of the adapter input (1 = kept)."""
+    keep = np.zeros((M, K), np.uint8)
+    _load().oracle_dropout_keep(M, K, dropout_threshold(p), seed, offset, _p(keep))
+    return keep
+
+
+def dropout_scale(p: float) -> float:
+    """1 / (1 - p) as the fp32 value both sides use."""
+    return float(np.float32(1.0 / (1.0 - p)))
+
+
+def linear_fwd_dropout(X, W, A, B, alpha: float, keep, p: float, rows=None):
+    """Y = X W^T + s (Xd A^T) B^T and U = Xd A^T with Xd = X * keep / (1 - p), fp64
+    (the adapter input of the PEFT LoRA layer goes through dropout, the frozen path does not)."""
+    X, W, A, B = (np.asarray(a, np.float64) for a in (X, W, A, B))
+    s = alpha / A.shape[0]
+    sel = slice(None) if rows is None else rows
+    Xd = X[sel] * keep[sel] * dropout_scale(p)
+    U = Xd @ A.T
+    return X[sel] @ W.T + s * U @ B.T, U
+
+
+def linear_bwd_dropout(X, W, A, B, dY, alpha: float, keep, p: float, rows=None):
+    """dX = dY W + s ((dY B) A) * keep / (1 - p), dA = s (dY B)^T Xd, dB = s dY^T (Xd A^T), fp64."""
+    X, W, A, B, dY = (np.asarray(a, np.float64) for a in (X, W, A, B, dY))
+    s = alpha / A.shape[0]
+    inv = dropout_scale(p)
+    Xd = X * keep * inv
+    V = dY @ B
+    sel = slice(None) if rows is None else rows
+    dX = dY[sel] @ W + s * (V[sel] @ A) * keep[sel] * inv
+    return dX, s * V.T @ Xd, s * dY.T @ (Xd @ A.T)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -359,6 +359,51 @@ void oracle_merge_adapter(const float* W, int64_t N, int64_t K, const uint16_t* 
 }
 
 /* ------------------------------------------------------------------------ */
+/* LoRA dropout on the adapter input ([p1] PEFT listing LoraConfig(...,     */
+/* lora_dropout=0.05); the adapter sees dropout(x) = x * keep / (1 - p)).    */
+/* The keep decisions come from Philox4x32-10, the counter-based generator  */
+/* of Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As Easy as   */
+/* 1, 2, 3" (SC'11), written here from that definition: 10 rounds of two    */
+/* 32x32->64 multiplications (multipliers 0xD2511F53, 0xCD9E8D57) with the  */
+/* key bumped by the Weyl constants (0x9E3779B9, 0xBB67AE85) between rounds. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c3 ^ k1;
+        uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Keep decision of element e (row-major index m*K + k of X): word (e & 3)  */
+/* of Philox4x32-10 with counter (lo32(e>>2), hi32(e>>2), lo32(offset),     */
+/* hi32(offset)) and key (lo32(seed), hi32(seed)); the element is kept when */
+/* that word is >= t, t = floor(p * 2^32) (the caller's integer threshold). */
+void oracle_dropout_keep(int64_t M, int64_t K, uint32_t t, uint64_t seed, uint64_t offset, uint8_t* keep) {
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+#pragma omp parallel for schedule(static)
+    for (int64_t q = 0; q < (M * K + 3) / 4; ++q) {
+        uint32_t ctr[4] = {(uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)offset, (uint32_t)(offset >> 32)};
+        uint32_t w[4];
+        oracle_philox4x32_10(ctr, key, w);
+        for (int j = 0; j < 4; ++j) {
+            int64_t e = q * 4 + j;
+            if (e < M * K) keep[e] = w[j] >= t ? 1 : 0;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* The linear layer in fp64, row-major.  W is N x K (out x in), X is M x K,  */
 /* A is r x K, B is N x r, s = alpha / r.                                    */
 /* [p1] "LoRAの復習" h = W0 x + (alpha/r) B A x, and "QLoRAの計算フロー"     */

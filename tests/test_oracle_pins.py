@@ -516,6 +516,64 @@ def test_merge_adapter_layer_identity():
     assert np.all(np.abs(got - ref) <= bound + 1e-12)
 
 
+# ------------------------------------------------------------- LoRA dropout
+def test_philox_known_answers():
+    kat = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.json")))
+    for v in kat["vectors"]:
+        h = lambda xs: np.array([int(x, 16) for x in xs], np.uint32)
+        assert np.array_equal(oracle.philox4x32_10(h(v["counter"]), h(v["key"])), h(v["out"]))
+
+
+def test_dropout_keep_rate_and_layout():
+    M, K = 512, 2048
+    for p in (0.05, 0.5):
+        keep = oracle.dropout_keep(M, K, p, seed=1234, offset=7)
+        n = keep.size
+        assert abs(keep.mean() - (1 - p)) <= 5 * np.sqrt(p * (1 - p) / n)
+    assert np.all(oracle.dropout_keep(8, 64, 0.0, seed=1, offset=0) == 1)
+    # element e = m*K + k uses word e & 3 of the block at counter (e >> 2, offset)
+    keep = oracle.dropout_keep(4, 64, 0.25, seed=0x1122334455667788, offset=0x99)
+    t = oracle.dropout_threshold(0.25)
+    for e in (0, 1, 2, 3, 4, 77, 255):
+        w = oracle.philox4x32_10([e >> 2, 0, 0x99, 0], [0x55667788, 0x11223344])
+        assert keep.reshape(-1)[e] == (1 if w[e & 3] >= t else 0)
+    # another offset gives another mask
+    assert not np.array_equal(oracle.dropout_keep(64, 64, 0.5, 3, 0), oracle.dropout_keep(64, 64, 0.5, 3, 1))
+
+
+def test_dropout_with_p_zero_is_the_plain_layer():
+    X, W, A, B, dY = _small_case()
+    keep = np.ones_like(X, dtype=np.uint8)
+    Y0, U0 = oracle.linear_fwd(X, W, A, B, 5.0)
+    Y1, U1 = oracle.linear_fwd_dropout(X, W, A, B, 5.0, keep, 0.0)
+    assert np.allclose(Y0, Y1, rtol=1e-13, atol=1e-13) and np.allclose(U0, U1, rtol=1e-13, atol=1e-13)
+    for a, b in zip(oracle.linear_bwd(X, W, A, B, dY, 5.0), oracle.linear_bwd_dropout(X, W, A, B, dY, 5.0, keep, 0.0)):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_dropout_bwd_against_finite_differences():
+    """With the mask fixed, L = <dY, Y> is smooth in A, B and X: central differences
+    check every gradient formula, including the masked adapter term of dX."""
+    X, W, A, B, dY = _small_case(M=6, N=10, K=64, r=3, seed=4)
+    p = 0.3
+    keep = oracle.dropout_keep(6, 64, p, seed=9, offset=0)
+    alpha = 4.0
+    L = lambda X_, A_, B_: float(np.sum(dY * oracle.linear_fwd_dropout(X_, W, A_, B_, alpha, keep, p)[0]))
+    dX, dA, dB = oracle.linear_bwd_dropout(X, W, A, B, dY, alpha, keep, p)
+    h = 1e-6
+    for name, arr, grad in (("A", A, dA), ("B", B, dB), ("X", X, dX)):
+        g = np.random.default_rng(0)
+        for _ in range(12):
+            idx = tuple(g.integers(0, d) for d in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args = {"A": (X, plus, B), "B": (X, A, plus), "X": (plus, A, B)}[name]
+            argm = {"A": (X, minus, B), "B": (X, A, minus), "X": (minus, A, B)}[name]
+            num = (L(*args) - L(*argm)) / (2 * h)
+            assert abs(num - grad[idx]) <= 1e-6 * max(1.0, abs(num)), (name, idx, num, grad[idx])
+
+
 # ----------------------------------------------------------------- linear
 def _small_case(M=9, N=24, K=64, r=3, seed=0):
     g = np.random.default_rng(seed)
