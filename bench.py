@@ -483,6 +483,40 @@ def run_merge(q, dev, peaks, reps=10):
             "requantize_ms": q_ms, "requantize_gbs": quant_bytes(N, K) / (q_ms * 1e-3) / 1e9}
 
 
+def run_dropout(q, dev, peaks, p=0.05, reps=10):
+    """The train4096 step's fwd+bwd with LoRA dropout p on the adapter input (the mask, a
+    masked adapter term of dX and the masked dA come on top of the plain step's work)."""
+    import torch
+    N, K, M, r, alpha = N_OUT, K_IN, M_TOK, RANK, ALPHA
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(gpu_weight(gen, N, K, "normal", dev))
+    X = torch.randn(M, K, generator=gen, device=dev).bfloat16()
+    A = (torch.randn(r, K, generator=gen, device=dev) / K ** 0.5).bfloat16()
+    B = (torch.randn(N, r, generator=gen, device=dev) * 0.01).bfloat16()
+    dY = torch.randn(M, N, generator=gen, device=dev).bfloat16()
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qlora_workspace_bytes_dropout(M, N, K, r), dtype=torch.uint8, device=dev)
+    it = [0]
+
+    def step():
+        it[0] += 1   # a fresh mask every step: offset = step index
+        q.qlora_linear_fwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, 1234, it[0], Y=Y, U_save=U, workspace=ws)
+        q.qlora_linear_bwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, 1234, it[0], dY, U_saved=U, dX=dX, dA=dA,
+                                   dB=dB, workspace=ws)
+
+    ms = time_region(step, 3, reps)
+    rc = q.qlora_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the dropout region: {q.qlora_strerror(rc)}")
+    return {"workload": f"train4096 layer fwd+bwd with LoRA dropout p={p} on the adapter input",
+            "fwd_bwd_ms": ms, "fwd_bwd_tflops": step_flops(M, N, K, r) / (ms * 1e-3) / 1e12}
+
+
 def run_configs(q, dev, peaks):
     import torch
     out = {"data": "seeded synthetic, generated on the GPU (torch generator) with the distributions named "
@@ -498,6 +532,8 @@ def run_configs(q, dev, peaks):
     out["train4096_fp8_dq"] = run_quant_variant(q, dev, peaks, "fp8")
     torch.cuda.empty_cache()
     out["train4096_merge_requantize"] = run_merge(q, dev, peaks)
+    torch.cuda.empty_cache()
+    out["train4096_dropout"] = run_dropout(q, dev, peaks)
     torch.cuda.empty_cache()
     return out
 

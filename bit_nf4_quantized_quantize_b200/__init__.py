@@ -16,10 +16,13 @@ from ._binding import (  # noqa: F401
     lib_path,
     load,
     qlora_dequant,
+    qlora_dropout_apply,
     qlora_launch_count,
     qlora_device_status,
     qlora_linear_bwd,
+    qlora_linear_bwd_dropout,
     qlora_linear_fwd,
+    qlora_linear_fwd_dropout,
     qlora_linear_fwd_noalloc,
     qlora_merge_adapter,
     qlora_nf4_codebook,
@@ -31,4 +34,5 @@ from ._binding import (  # noqa: F401
     qlora_timing_collect,
     qlora_timing_enable,
     qlora_workspace_bytes,
+    qlora_workspace_bytes_dropout,
 )

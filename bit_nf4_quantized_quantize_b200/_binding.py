@@ -50,6 +50,20 @@ _SIGNATURES = {
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "qlora_workspace_bytes_dropout": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
+    "qlora_linear_fwd_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                                ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_linear_bwd_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                                ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_dropout_apply": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
+                                           ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_selftest_device_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_timing_enable": (ctypes.c_int, [ctypes.c_int]),
     "qlora_timing_collect": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]),
@@ -57,7 +71,7 @@ _SIGNATURES = {
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "lora_gemm", "lora_reduce", "fwd_fused", "dx_fused", "grad_gemm",
-                "grad_reduce", "fwd_decode", "merge"]
+                "grad_reduce", "fwd_decode", "merge", "dropout"]
 
 
 class QloraError(RuntimeError):
@@ -309,6 +323,78 @@ def qlora_linear_bwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float
                                    ws.numel(), _stream(stream)),
            "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_workspace_bytes_dropout(M: int, n_out: int, k_in: int, r: int) -> int:
+    return int(load().qlora_workspace_bytes_dropout(M, n_out, k_in, r))
+
+
+def _workspace_dropout(ws, M, N, K, r, device):
+    need = qlora_workspace_bytes_dropout(M, N, K, r)
+    if need == 0:
+        raise QloraError(-2, "qlora_workspace_bytes_dropout")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def qlora_linear_fwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float, p: float, seed: int,
+                             offset: int, Y=None, U_save=None, workspace=None, stream=None):
+    """The forward with dropout p on the adapter input (Philox keep mask from seed, offset)."""
+    _weight(codes, q8, s2, n_out, k_in)
+    M = X.shape[0]
+    r = A.shape[0]
+    _dev(X, torch.bfloat16, "X", (M, k_in))
+    _dev(A, torch.bfloat16, "A", (r, k_in))
+    _dev(B, torch.bfloat16, "B", (n_out, r))
+    Y = torch.empty(M, n_out, dtype=torch.bfloat16, device=X.device) if Y is None else _dev(Y, torch.bfloat16, "Y", (M, n_out))
+    if U_save is not None:
+        _dev(U_save, torch.bfloat16, "U_save", (M, r))
+    ws = _workspace_dropout(workspace, M, n_out, k_in, r, X.device)
+    _check(load().qlora_linear_fwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
+                                           _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(Y),
+                                           _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_fwd_dropout")
+    return Y
+
+
+def qlora_linear_bwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float, p: float, seed: int,
+                             offset: int, dY, U_saved=None, dX=None, dA=None, dB=None, need_dX=True,
+                             workspace=None, stream=None):
+    """The backward with dropout p on the adapter input -> (dX or None, dA, dB)."""
+    _weight(codes, q8, s2, n_out, k_in)
+    M = X.shape[0]
+    r = A.shape[0]
+    _dev(X, torch.bfloat16, "X", (M, k_in))
+    _dev(A, torch.bfloat16, "A", (r, k_in))
+    _dev(B, torch.bfloat16, "B", (n_out, r))
+    _dev(dY, torch.bfloat16, "dY", (M, n_out))
+    if U_saved is not None:
+        _dev(U_saved, torch.bfloat16, "U_saved", (M, r))
+    dev = X.device
+    if need_dX:
+        dX = torch.empty(M, k_in, dtype=torch.bfloat16, device=dev) if dX is None else _dev(dX, torch.bfloat16, "dX", (M, k_in))
+    else:
+        dX = None
+    dA = torch.empty(r, k_in, dtype=torch.float32, device=dev) if dA is None else _dev(dA, torch.float32, "dA", (r, k_in))
+    dB = torch.empty(n_out, r, dtype=torch.float32, device=dev) if dB is None else _dev(dB, torch.float32, "dB", (n_out, r))
+    ws = _workspace_dropout(workspace, M, n_out, k_in, r, dev)
+    _check(load().qlora_linear_bwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
+                                           _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(dY),
+                                           _ptr(U_saved), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                                           _stream(stream)),
+           "qlora_linear_bwd_dropout")
+    return dX, dA, dB
+
+
+def qlora_dropout_apply(X, p: float, seed: int, offset: int, out=None, stream=None):
+    """X * keep (bf16, dropped elements 0): the masked adapter input of the dropout calls."""
+    M, K = X.shape
+    _dev(X, torch.bfloat16, "X", (M, K))
+    out = torch.empty_like(X) if out is None else _dev(out, torch.bfloat16, "out", (M, K))
+    _check(load().qlora_dropout_apply(_ptr(X), M, K, float(p), int(seed), int(offset), _ptr(out), _stream(stream)),
+           "qlora_dropout_apply")
+    return out
 
 
 def qlora_device_status(stream=None) -> int:

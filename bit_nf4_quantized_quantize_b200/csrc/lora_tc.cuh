@@ -30,9 +30,9 @@ constexpr int kLoraBN = 64;
 constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
 enum LoraOut : int {
-  kLoraOutPlainScaled = 0,  // bf16 out0 = sum (may be NULL), bf16 out1 = s * sum; row-major [rows][r]
-  kLoraOutTransposed = 1,   // fp32 out0[col][row] = s * sum  (dA from dA^T tiles)
-  kLoraOutRowMajor = 2,     // fp32 out0[row][col] = s * sum  (dB)
+  kLoraOutPlainScaled = 0,  // bf16 out0 = scale0 * sum (may be NULL), bf16 out1 = scale1 * sum; [rows][r]
+  kLoraOutTransposed = 1,   // fp32 out0[col][row] = scale1 * sum  (dA from dA^T tiles)
+  kLoraOutRowMajor = 2,     // fp32 out0[row][col] = scale1 * sum  (dB)
 };
 
 struct LoraProblem {
@@ -45,13 +45,14 @@ struct LoraProblem {
   void* out0;
   void* out1;
   int ld_t;        // kLoraOutTransposed: elements between out0 rows (= rows)
+  float scale0;    // kLoraOutPlainScaled: factor of out0 (1 for U or V itself)
+  float scale1;    // factor of out1 (PlainScaled) or of out0 (fp32 outputs)
 };
 
 struct LoraArgs {
   LoraProblem p[2];
   int tiles0;      // blocks of problem 0 along x (tiles_m * tiles_n)
   int r;
-  float s;
 };
 
 struct LoraSmem {
@@ -221,11 +222,13 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
       const int grow = m0 + trow;
       const int gcol = c0 + c16 * 4;
       if (grow < P.rows && gcol < args.r) {
-        const float s = args.s;
+        const float s = P.scale1;
         if (P.out_kind == kLoraOutPlainScaled) {
           const int64_t o = static_cast<int64_t>(grow) * args.r + gcol;
           if (P.out0) {
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y), h1 = __floats2bfloat162_rn(acc.z, acc.w);
+            const float s0 = P.scale0;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(s0 * acc.x, s0 * acc.y);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(s0 * acc.z, s0 * acc.w);
             uint2 u;
             u.x = *reinterpret_cast<uint32_t*>(&h0);
             u.y = *reinterpret_cast<uint32_t*>(&h1);

@@ -26,6 +26,7 @@
 #include "fused2_tc.cuh"
 #include "decode_tc.cuh"
 #include "merge.cuh"
+#include "dropout.cuh"
 
 using namespace qlora;
 
@@ -374,20 +375,22 @@ int run_decode(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t us, v, vs, u, total;
+  size_t us, v, vs, u, xm, total;
 };
 
 // bf16 scratch of M x r each: s*U (forward adapter operand), V and s*V
 // (backward), U (recomputed when the caller passes no saved U).
-WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms) {
-  (void)N; (void)K; (void)num_sms;
+// With dropout, xm holds the masked adapter input X * keep (bf16 M x K).
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms, bool dropout = false) {
+  (void)N; (void)num_sms;
   WsLayout w;
   const size_t mr = a256(static_cast<size_t>(M) * r * 2);
   w.us = 0;
   w.v = w.us + mr;
   w.vs = w.v + mr;
   w.u = w.vs + mr;
-  w.total = w.u + mr;
+  w.xm = w.u + mr;
+  w.total = w.xm + (dropout ? a256(static_cast<size_t>(M) * K * 2) : 0);
   return w;
 }
 
@@ -478,8 +481,11 @@ int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap&
   });
 }
 
-LoraProblem lora_problem(int rows, int k_steps, int S, int rpad, int kind, void* out0, void* out1, int ld_t) {
+LoraProblem lora_problem(int rows, int k_steps, int S, int rpad, int kind, void* out0, void* out1, int ld_t,
+                         float scale0, float scale1) {
   LoraProblem p{};
+  p.scale0 = scale0;
+  p.scale1 = scale1;
   p.rows = rows;
   p.k_steps = k_steps;
   p.per_split = (k_steps + S - 1) / S;
@@ -515,8 +521,8 @@ void fill_levels(GemmArgs& g) {
   for (int i = 0; i < 16; ++i) g.level[i] = tables().level[i];
 }
 
-// U = X A^T into `plain` (bf16, may be NULL) and `scaled` = bf16(s U) (may be NULL).
-int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat, int r, float s,
+// acc = X A^T; `plain` = bf16(scale0 acc) and `scaled` = bf16(scale1 acc), each may be NULL.
+int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat, int r, float scale0, float scale1,
                   uint16_t* plain, uint16_t* scaled, int num_sms, cudaStream_t st, int dev) {
   const int rpad = (r + 63) / 64 * 64;
   CUtensorMap ta, tb;
@@ -525,12 +531,48 @@ int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat,
   const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
   const int S = lora_cluster(tiles, k_steps, num_sms);
   LoraArgs la{};
-  la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, plain, scaled, 0);
+  la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, plain, scaled, 0, scale0,
+                         scale1);
   la.p[1] = la.p[0];
   la.tiles0 = tiles;
   la.r = r;
-  la.s = s;
   return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM);
+}
+
+// ------------------------------------------------------------------ LoRA dropout
+// Dropout on the adapter input (dropout.cuh): integer keep threshold t =
+// floor(p * 2^32) and scale inv = fp32(1 / (1 - p)), both from the fp32 p.
+struct DropoutSpec {
+  bool on = false;
+  uint32_t t = 0;
+  float inv = 1.f;
+  uint64_t seed = 0, offset = 0;
+};
+
+// Returns false if p is not in [0, 1).  p == 0 leaves the spec off.
+bool make_dropout(float p, uint64_t seed, uint64_t offset, DropoutSpec* d) {
+  if (!(p >= 0.f && p < 1.f)) return false;
+  *d = DropoutSpec{};
+  if (p == 0.f) return true;
+  const double pd = static_cast<double>(p);
+  const double tt = std::floor(pd * 4294967296.0);
+  d->on = true;
+  d->t = tt >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(tt);
+  d->inv = static_cast<float>(1.0 / (1.0 - pd));
+  d->seed = seed;
+  d->offset = offset;
+  return true;
+}
+
+// X * keep (bf16 M x K) into `out`.
+int launch_dropout_mask(const uint16_t* X, int64_t M, int64_t K, const DropoutSpec& d, uint16_t* out, int sms,
+                        cudaStream_t st) {
+  const int64_t n4 = M * K / 4;
+  const int64_t want = (n4 + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  return timed(QLORA_KERNEL_DROPOUT, st, [&] {
+    return launch_ex(dropout_mask_kernel, dim3(blocks), dim3(256), 0, st, 1, 1, X, n4, d.t, d.seed, d.offset, out);
+  });
 }
 
 // ------------------------------------------------------------------ failure-path self-test
@@ -713,16 +755,18 @@ size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r) {
   return ws_layout(M, n_out, k_in, r, sms).total;
 }
 
-int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
-                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
-                     uint16_t* Y, uint16_t* U_save, void* workspace, size_t workspace_bytes, void* stream) {
+// The forward with (dr.on) or without dropout on the adapter input.
+static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                    const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                    uint16_t* Y, uint16_t* U_save, void* workspace, size_t workspace_bytes, void* stream,
+                    const DropoutSpec& dr) {
   if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
   if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
   if (!Y) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
-  const WsLayout L = ws_layout(M, n_out, k_in, r, sms);
+  const WsLayout L = ws_layout(M, n_out, k_in, r, sms, dr.on);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -732,10 +776,17 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   const int rpad = (r + 63) / 64 * 64;
 
   // a few tokens: one launch, weight rows on the MMA's M side, U computed in-kernel
-  if (M <= kDecMaxTokens && r <= kDecMaxRank)
+  if (M <= kDecMaxTokens && r <= kDecMaxRank && !dr.on)
     return run_decode(codes, q8, s2, n_out, k_in, X, M, A, B, r, s, Y, U_save, st, dev);
 
-  if (int rc = run_lora_down(X, M, k_in, A, r, s, U_save, Us, sms, st, dev)) return rc;
+  if (dr.on) {
+    // the adapter's input goes through dropout: U = (X * keep) A^T / (1 - p)
+    uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
+    if (int rc = launch_dropout_mask(X, M, k_in, dr, Xm, sms, st)) return rc;
+    if (int rc = run_lora_down(Xm, M, k_in, A, r, dr.inv, s * dr.inv, U_save, Us, sms, st, dev)) return rc;
+  } else if (int rc = run_lora_down(X, M, k_in, A, r, 1.f, s, U_save, Us, sms, st, dev)) {
+    return rc;
+  }
 
   GemmArgs g{};
   g.m_rows = static_cast<int>(M);
@@ -779,6 +830,23 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
   return launch_gemm<256, 4, false, kBDeqK, kOutBf16, 8, 1>(grid, tx, tp, tus, tb, g, st, dev);
 }
 
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* Y, uint16_t* U_save, void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, Y, U_save, workspace, workspace_bytes, stream,
+                  DropoutSpec{});
+}
+
+int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                             const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             float p, uint64_t seed, uint64_t offset, uint16_t* Y, uint16_t* U_save, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  DropoutSpec dr;
+  if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  return fwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, Y, U_save, workspace, workspace_bytes, stream,
+                  dr);
+}
+
 // Forward with the library's own fixed scratch instead of a caller workspace:
 // for callers that cannot allocate device memory (see include/qlora_nf4.h).
 int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out,
@@ -797,10 +865,11 @@ int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const floa
                           kNoAllocScratchBytes, stream);
 }
 
-int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
-                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
-                     const uint16_t* dY, const uint16_t* U_saved, uint16_t* dX, float* dA, float* dB,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+// The backward with (dr.on) or without dropout on the adapter input.
+static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                    const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                    const uint16_t* dY, const uint16_t* U_saved, uint16_t* dX, float* dA, float* dB,
+                    void* workspace, size_t workspace_bytes, void* stream, const DropoutSpec& dr) {
   if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
   if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
   if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
@@ -809,7 +878,7 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
-  const WsLayout L = ws_layout(M, n_out, k_in, r, sms);
+  const WsLayout L = ws_layout(M, n_out, k_in, r, sms, dr.on);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -829,27 +898,35 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
     const int S = lora_cluster(tiles, k_steps, sms);
     LoraArgs la{};
-    la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, V, Vs, 0);
+    la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, V, Vs, 0, 1.f, s);
     la.p[1] = la.p[0];
     la.tiles0 = tiles;
     la.r = r;
-    la.s = s;
     if (int rc = launch_lora<false, true>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM)) return rc;
+  }
+  // the adapter's input: X, or X * keep with dropout (the 1/(1-p) goes into the scales)
+  const uint16_t* Xa = X;
+  if (dr.on) {
+    uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
+    if (int rc = launch_dropout_mask(X, M, K, dr, Xm, sms, st)) return rc;
+    Xa = Xm;
   }
   // U (from the forward, or recomputed)
   const uint16_t* U = U_saved;
   if (!U) {
-    if (int rc = run_lora_down(X, M, K, A, r, s, Ubuf, nullptr, sms, st, dev)) return rc;
+    if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev)) return rc;
     U = Ubuf;
   }
-  // dX = dY dequant(W) + (s V) A
+  // dX = dY dequant(W) + (s V) A; with dropout the adapter term is masked, so
+  // the fused kernel computes dY dequant(W) alone and dropout_dx_kernel adds
+  // s/(1-p) (V A) where the input was kept
   if (dX) {
     GemmArgs g{};
     g.m_rows = static_cast<int>(M);
     g.n_cols = K;
     g.k_steps = N / 64;
     g.steps_per_split = g.k_steps;
-    g.n_lora = rpad / 64;
+    g.n_lora = dr.on ? 0 : rpad / 64;
     g.q8 = q8;
     g.s2 = s2;
     g.w_rows = N;
@@ -882,11 +959,23 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
       rc = launch_gemm<256, 4, false, kBDeqMN, kOutBf16, 8, 1>(grid, ta, tp, ta2, tb2, g, st, dev);
     }
     if (rc) return rc;
+    if (dr.on) {
+      const dim3 grid(static_cast<unsigned>((K + 4 * kDxThreads - 1) / (4 * kDxThreads)),
+                      static_cast<unsigned>((M + kDxRows - 1) / kDxRows));
+      const size_t smem = sizeof(float) * kDxRows * static_cast<size_t>(r);
+      const float scale = s * dr.inv;
+      rc = timed(QLORA_KERNEL_DROPOUT, st, [&] {
+        return launch_ex(dropout_dx_kernel, grid, dim3(kDxThreads), smem, st, 1, 1, dX, V, A, M,
+                         static_cast<int64_t>(K), r, scale, dr.t, dr.seed, dr.offset);
+      });
+      if (rc) return rc;
+    }
   }
-  // dA^T = X^T V and dB = dY^T U in one grouped launch, reduced over M
+  // dA^T = X^T V and dB = dY^T U in one grouped launch, reduced over M (X * keep and s/(1-p)
+  // for dA with dropout)
   {
     CUtensorMap ta0, tb0, ta1, tb1;
-    if (!map_bf16(&ta0, X, M, K, 64, 64) || !map_bf16(&tb0, V, M, r, 64, 64) ||
+    if (!map_bf16(&ta0, Xa, M, K, 64, 64) || !map_bf16(&tb0, V, M, r, 64, 64) ||
         !map_bf16(&ta1, dY, M, N, 64, 64) || !map_bf16(&tb1, U, M, r, 64, 64))
       return QLORA_ERR_CUDA;
     const int k_steps = static_cast<int>((M + 63) / 64);
@@ -894,16 +983,55 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
     const int tiles_b = ((N + 127) / 128) * (rpad / 64);
     const int S = lora_cluster(tiles_a + tiles_b, k_steps, sms);
     LoraArgs la{};
-    la.p[0] = lora_problem(K, k_steps, S, rpad, kLoraOutTransposed, dA, nullptr, K);
-    la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0);
+    la.p[0] = lora_problem(K, k_steps, S, rpad, kLoraOutTransposed, dA, nullptr, K, 1.f, s * dr.inv);
+    la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0, 1.f, s);
     la.tiles0 = tiles_a;
     la.r = r;
-    la.s = s;
     if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, st, dev,
                                          QLORA_KERNEL_GRAD_GEMM))
       return rc;
   }
   return QLORA_OK;
+}
+
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                     const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     const uint16_t* dY, const uint16_t* U_saved, uint16_t* dX, float* dA, float* dB,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, dY, U_saved, dX, dA, dB, workspace,
+                  workspace_bytes, stream, DropoutSpec{});
+}
+
+int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
+                             const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             float p, uint64_t seed, uint64_t offset, const uint16_t* dY, const uint16_t* U_saved,
+                             uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  DropoutSpec dr;
+  if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  return bwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, dY, U_saved, dX, dA, dB, workspace,
+                  workspace_bytes, stream, dr);
+}
+
+size_t qlora_workspace_bytes_dropout(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 1 || n_out < 64 || k_in < 64 || r < 1 || r > 256) return 0;
+  int dev = 0, sms = 148;
+  if (check_device(&dev, &sms) != QLORA_OK) sms = 148;
+  return ws_layout(M, n_out, k_in, r, sms, true).total;
+}
+
+int qlora_dropout_apply(const uint16_t* X, int64_t M, int64_t k_in, float p, uint64_t seed, uint64_t offset,
+                        uint16_t* out, void* stream) {
+  if (!X || !out) return QLORA_ERR_INVALID_ARG;
+  if (M < 1 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  DropoutSpec dr;
+  if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!dr.on) dr.t = 0;   // p == 0: every element kept (the same kernel, threshold 0)
+  return launch_dropout_mask(X, M, k_in, dr, out, sms, st);
 }
 
 int64_t qlora_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }

@@ -237,6 +237,53 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * LoRA dropout on the adapter input ("QLoRAの理論と実装", PEFT listing:
+ * LoraConfig(..., lora_dropout=0.05)).  The adapter sees x * keep / (1 - p);
+ * the frozen NF4 path sees x:
+ *   Y  = X dequant(W)^T + s (Xd A^T) B^T,  U = Xd A^T,  Xd = X * keep / (1 - p)
+ *   dX = dY dequant(W) + s ((dY B) A) * keep / (1 - p)
+ *   dA = s (dY B)^T Xd,  dB = s dY^T U
+ * keep(e) for element e = m*K + k of X: word (e & 3) of Philox4x32-10 (Salmon
+ * et al., SC'11) at counter (lo32(e>>2), hi32(e>>2), lo32(offset),
+ * hi32(offset)) with key (lo32(seed), hi32(seed)) is >= floor(p * 2^32); the
+ * scale is fp32(1 / (1 - p)); both are taken from the fp32 p.  p must be in
+ * [0, 1) (else QLORA_ERR_INVALID_ARG); p == 0 is exactly the plain call.
+ * Pass the same (p, seed, offset) to the forward and the backward of a step.
+ * The workspace must hold qlora_workspace_bytes_dropout(M, N, K, r) bytes
+ * (the plain size plus a bf16 M x K masked copy of X).  Arguments otherwise
+ * as qlora_linear_fwd / qlora_linear_bwd.  Launches: mask, U, the fused
+ * GEMM (forward); mask, V, [U], dY dequant(W), the masked adapter term of dX,
+ * dA/dB (backward).  M <= 32 takes the tiled path (the few-token kernel
+ * forms U from the unmasked tile).
+ */
+size_t qlora_workspace_bytes_dropout(int64_t M, int64_t n_out, int64_t k_in, int r);
+
+int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                             int64_t n_out, int64_t k_in,
+                             const uint16_t* X, int64_t M,
+                             const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             float p, uint64_t seed, uint64_t offset,
+                             uint16_t* Y, uint16_t* U_save,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2,
+                             int64_t n_out, int64_t k_in,
+                             const uint16_t* X, int64_t M,
+                             const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             float p, uint64_t seed, uint64_t offset,
+                             const uint16_t* dY, const uint16_t* U_saved,
+                             uint16_t* dX, float* dA, float* dB,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The masked adapter input of the dropout calls: out = X * keep (bf16 M x K,
+ * dropped elements +0; the 1/(1 - p) is not applied).  For tests and export;
+ * the dropout calls form it in their workspace.  One kernel launch.
+ */
+int qlora_dropout_apply(const uint16_t* X, int64_t M, int64_t k_in, float p, uint64_t seed,
+                        uint64_t offset, uint16_t* out, void* stream);
+
+/*
  * Diagnostic for the failure path.  Enqueues one warp that waits, bounded, on
  * an mbarrier nothing arrives at: the wait gives up after the library's limit
  * (2 s of %globaltimer), latches the device error flag exactly as an expired
@@ -275,7 +322,8 @@ int qlora_device_status(void* stream);
 #define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
 #define QLORA_KERNEL_FWD_DECODE 8  /* small-M forward (M <= 32, r <= 64)     */
 #define QLORA_KERNEL_MERGE 9       /* adapter merge into the 16-bit base      */
-#define QLORA_KERNEL_COUNT 10
+#define QLORA_KERNEL_DROPOUT 10    /* dropout mask / masked adapter dX        */
+#define QLORA_KERNEL_COUNT 11
 int qlora_timing_enable(int on);
 /* Number of kernels the library has enqueued since it was loaded (all
  * devices, all streams), counted whether or not timing is enabled. */

@@ -235,10 +235,12 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 
 def dropout_threshold(p: float) -> int:
-    """Integer keep threshold floor(p * 2^32) (clamped to 2^32 - 1); element kept iff its word >= it."""
-    if not 0.0 <= p < 1.0:
+    """Integer keep threshold floor(p * 2^32) of the fp32 value of p (clamped to 2^32 - 1);
+    an element is kept iff its word >= it."""
+    p32 = float(np.float32(p))
+    if not 0.0 <= p32 < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(int(np.floor(p * 4294967296.0)), 0xFFFFFFFF)
+    return min(int(np.floor(p32 * 4294967296.0)), 0xFFFFFFFF)
 
 
 def dropout_keep(M: int, K: int, p: float, seed: int, offset: int) -> np.ndarray:
@@ -249,8 +251,8 @@ def dropout_keep(M: int, K: int, p: float, seed: int, offset: int) -> np.ndarray
 
 
 def dropout_scale(p: float) -> float:
-    """1 / (1 - p) as the fp32 value both sides use."""
-    return float(np.float32(1.0 / (1.0 - p)))
+    """1 / (1 - p) of the fp32 value of p, rounded to fp32: the value both sides use."""
+    return float(np.float32(1.0 / (1.0 - float(np.float32(p)))))
 
 
 def linear_fwd_dropout(X, W, A, B, alpha: float, keep, p: float, rows=None):
