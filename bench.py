@@ -47,6 +47,23 @@ def step_flops(M, N, K, r):
     return 4 * M * N * K + 2 * M * r * (K + N) + 2 * M * r * (N + K) + 2 * r * M * K + 2 * N * M * r
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (every rank gets it); x itself on one rank.  Times of a
+    multi-GPU run are the slowest rank's."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, ms: float, scale: float = 1e12) -> float:
+    """Whole-job rate: the units all ranks processed (replicas: world x per rank) / the step time."""
+    return world * units_per_rank / (ms * 1e-3) / scale
+
+
 def quant_bytes(N, K):
     """Algorithmic quantize traffic: fp32 W in, packed codes + q8 + s2 out."""
     n = N * K
@@ -635,11 +652,7 @@ def run_ours(args, rank, world, local_rank):
     rc = q.qlora_device_status()
     if rc != 0:
         raise RuntimeError(f"device status after the timed region: {q.qlora_strerror(rc)}")
-    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world, dev)
 
     # ---------------------------------------------------------------- per-kernel breakdown
     # The same steps again with a CUDA event pair around every library launch
@@ -684,16 +697,12 @@ def run_ours(args, rank, world, local_rank):
         hdB.copy_(dB, non_blocking=True)
         e_ev[i][1].record()
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e_ev) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / n_e2e, world, dev)
 
     if rank != 0:
         return
     fl = step_flops(M, N, K, r)
-    value = world * fl / (step_ms * 1e-3) / 1e12
+    value = job_throughput(world, fl, step_ms)
     peaks = load_peaks()
     per_step = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps,
                     "ms_per_launch": v[0] / v[1]} for k, v in kern.items()}
@@ -731,7 +740,7 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes": quant_bytes(N, K), "traffic": load_traffic("quantize")},
         "kernels": per_step,
         "gpu_launches": launches,
-        "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(world, fl, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "clocks": clocks,
     }
