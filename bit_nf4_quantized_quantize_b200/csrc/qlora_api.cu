@@ -56,7 +56,7 @@ double normal_quantile(double p) {
 // Decision thresholds: code(n) = #{i : n > (level_i + level_{i+1})/2}, the
 // exact nearest level with the lower index on a tie; thr_i is the smallest
 // fp32 above that exact midpoint, so code(n) = #{i : n >= thr_i}.  The
-// 257-cell table indexes floor(128 n) + 128 for n in [-1, 1].
+// 33-cell table indexes floor(16 n) + 16 for n in [-1, 1].
 Nf4Tables build_tables() {
   Nf4Tables T;
   std::memset(&T, 0, sizeof(T));

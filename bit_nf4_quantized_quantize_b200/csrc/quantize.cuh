@@ -18,7 +18,12 @@
 // the smallest fp32 above the exact midpoint of levels i and i+1.  Cells of
 // width 1/16 over [-1, 1] hold at most one threshold each (the thresholds are
 // >= 0.088 apart), so code = lo[cell] + (n >= thr[cell]) with cell =
-// floor(16 n) + 16.  Fast path: q0 = fp32(w * fp32(1/absmax)) is within 2.5
+// floor(16 n) + 16.  The cell comes from the float adder rather than a
+// conversion: u = fp32(fp32(16 n + 15.5) + 1.5 * 2^23) lies in the binade of
+// ulp 1, whose low 6 mantissa bits are then RN(16 n + 15.5) = floor(16 n + 16)
+// away from the cell edges; within 2^-17 of an edge the cell may be the left
+// or right neighbour, which decides the same code because no threshold lies
+// within 2^-17 of an edge (the host checks this).  Fast path: q0 = fp32(w * fp32(1/absmax)) is within 2.5
 // ulp of n, so every threshold that is not within 2^-18 of q0 lies on the
 // same side of q0 and n; the fast table packs the cell's left-edge code into
 // the 4 low mantissa bits of its threshold (a perturbation below 2^-19) and
@@ -37,6 +42,7 @@ namespace qlora {
 constexpr int kBlock = 64;     // first-level block
 constexpr int kGroup = 256;    // second-level group (blocks per s2)
 constexpr int kLutCells = 33;  // floor(16 n) + 16 for n in [-1, 1]
+constexpr int kLutPad = 64;    // table entries in shared memory: any 6-bit index is in range
 constexpr float kFastGuard = 3.814697265625e-06f;  // 2^-18
 
 // Host-built tables handed to the kernels by value.
@@ -60,15 +66,17 @@ template <int kMode>
 __global__ void __launch_bounds__(kQuantThreads, 2)
 quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
                     uint8_t* __restrict__ q8, float* __restrict__ s2, const Nf4Tables tabs) {
-  __shared__ int2 s_exact[kLutCells];     // {threshold bits, left-edge code}
-  __shared__ uint32_t s_fast[kLutCells];
+  __shared__ int2 s_exact[kLutPad];     // {threshold bits, left-edge code}
+  __shared__ uint32_t s_fast[kLutPad];
   __shared__ float s_absmax[kGroup];
   __shared__ float s_warpmax[kGroup / 32];
 
   const int tid = threadIdx.x;
-  if (tid < kLutCells) {
-    s_exact[tid] = make_int2(__float_as_int(tabs.cell_thr[tid]), tabs.cell_lo[tid]);
-    s_fast[tid] = tabs.cell_fast[tid];
+  if (tid < kLutPad) {
+    // entries past the last cell repeat it (only NaN input, a caller error, reaches them)
+    const int c = tid < kLutCells ? tid : kLutCells - 1;
+    s_exact[tid] = make_int2(__float_as_int(tabs.cell_thr[c]), tabs.cell_lo[c]);
+    s_fast[tid] = tabs.cell_fast[c];
   }
   const bool fast_table = tabs.fast_ok != 0;
 
@@ -108,34 +116,41 @@ quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, uint8_t* __re
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
-    if (lb < nb) {
-      // fast path needs fp32(1/absmax) to be a normal number
-      const bool fast = fast_table && am >= 2.35098870e-38f * 4.0f && am <= 4.2535296e37f;
-      const float rcp = fast ? __frcp_rn(am) : 0.f;
-      uint32_t packed = 0;
+    // every lane takes part (the warp-wide vote below); blocks past the end hold
+    // zeros and are not stored
+    // fast path needs fp32(1/absmax) to be a normal number
+    const bool fast = fast_table && am >= 2.35098870e-38f * 4.0f && am <= 4.2535296e37f;
+    uint32_t packed = 0x88888888u;   // an all-zero block: every code is 8 (the level 0.0)
+    uint32_t slow = 0;               // weights the fast path cannot decide
+    if (fast) {
+      const float rcp = __frcp_rn(am);
+      packed = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        int code;
-        bool exact = !fast;
-        if (fast) {
-          const float q0 = __fmul_rn(e[j], rcp);
-          const unsigned cell = min(static_cast<unsigned>(__float2int_rd(q0 * 16.f) + 16), 32u);
-          const uint32_t ent = s_fast[cell];
-          const float thr = __uint_as_float(ent);
-          code = static_cast<int>(ent & 15u) + (q0 >= thr ? 1 : 0);
-          exact = fabsf(q0 - thr) <= kFastGuard;
-        }
-        if (exact) {
-          // one IEEE fp32 division, round to nearest (never the reciprocal form)
-          const float wn = am > 0.f ? __fdiv_rn(e[j], am) : 0.f;
-          // |wn| <= 1, so floor(16 wn) + 16 is in [0, 32]; the unsigned min
-          // only guards against NaN input (a caller error)
-          const unsigned cell = min(static_cast<unsigned>(__float2int_rd(wn * 16.f) + 16), 32u);
-          const int2 ent = s_exact[cell];
-          code = ent.y + (wn >= __int_as_float(ent.x) ? 1 : 0);
-        }
-        packed |= static_cast<uint32_t>(code) << (4 * j);
+        const float q0 = __fmul_rn(e[j], rcp);
+        const uint32_t cell = __float_as_uint(__fadd_rn(__fmaf_rn(q0, 16.f, 15.5f), 12582912.f)) & 63u;
+        const uint32_t ent = s_fast[cell];
+        const float thr = __uint_as_float(ent);
+        packed |= ((ent & 15u) + (q0 >= thr ? 1u : 0u)) << (4 * j);
+        slow |= (fabsf(q0 - thr) <= kFastGuard ? 1u : 0u) << j;
       }
+    } else if (am > 0.f) {
+      slow = 0xFFu;
+    }
+    if (__any_sync(0xffffffffu, slow != 0u)) {
+      // one IEEE fp32 division per undecided weight, round to nearest (never the reciprocal form)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if ((slow >> j) & 1u) {
+          const float wn = __fdiv_rn(e[j], am);
+          const uint32_t cell = __float_as_uint(__fadd_rn(__fmaf_rn(wn, 16.f, 15.5f), 12582912.f)) & 63u;
+          const int2 ent = s_exact[cell];
+          const uint32_t code = static_cast<uint32_t>(ent.y) + (wn >= __int_as_float(ent.x) ? 1u : 0u);
+          packed = (packed & ~(15u << (4 * j))) | (code << (4 * j));
+        }
+      }
+    }
+    if (lb < nb) {
       *reinterpret_cast<uint32_t*>(codes + ((b_first + lb) * kBlock + sub * 8) / 2) = packed;
       if (sub == 0) {
         if (kMode != kQuantSingle) s_absmax[lb] = am;
