@@ -69,35 +69,36 @@ Nf4Tables build_tables() {
   for (double a : v) mx = std::max(mx, std::fabs(a));
   for (int i = 0; i < 16; ++i) T.level[i] = static_cast<float>(v[i] / mx);
   std::sort(T.level, T.level + 16);
+  double mid[15];
   float thr[15];
   for (int i = 0; i < 15; ++i) {
-    const double mid = (static_cast<double>(T.level[i]) + static_cast<double>(T.level[i + 1])) * 0.5;
-    float f = static_cast<float>(mid);
-    if (static_cast<double>(f) <= mid) f = std::nextafter(f, INFINITY);
+    mid[i] = (static_cast<double>(T.level[i]) + static_cast<double>(T.level[i + 1])) * 0.5;
+    float f = static_cast<float>(mid[i]);
+    if (static_cast<double>(f) <= mid[i]) f = std::nextafter(f, INFINITY);
     thr[i] = f;
   }
   // cells of width 1/16: cell c covers [(c-16)/16, (c-15)/16)
   T.fast_ok = 1;
   for (int c = 0; c < kLutCells; ++c) {
     const double lo = (c - 16) / 16.0, hi = (c - 15) / 16.0;
-    int cnt = 0, inside_n = 0;
-    float inside = INFINITY;
+    int cnt = 0, inside_n = 0, inside_i = -1;
     for (int i = 0; i < 15; ++i) {
-      if (thr[i] <= lo) ++cnt;
-      else if (thr[i] < hi) { inside = std::min(inside, thr[i]); ++inside_n; }
+      if (mid[i] < lo) ++cnt;
+      else if (mid[i] < hi) { if (inside_i < 0) inside_i = i; ++inside_n; }
     }
     T.cell_lo[c] = cnt;
-    T.cell_thr[c] = inside;
-    if (inside_n > 1) T.fast_ok = 0;  // (cannot happen for this table: thresholds are >= 0.088 apart)
-    // fast entry: threshold (4.0 when the cell has none) with the code in its 4 low bits
+    T.cell_thr[c] = inside_i < 0 ? INFINITY : thr[inside_i];
+    if (inside_n > 1) T.fast_ok = 0;  // (cannot happen for this table: midpoints are >= 0.088 apart)
+    // fast entry, in units of t = 16 n + 15.875: the midpoint (64.0 when the
+    // cell has none, above every t) with the code in its 4 low mantissa bits
+    const float f = inside_i < 0 ? 64.0f : static_cast<float>(16.0 * mid[inside_i] + 15.875);
     uint32_t bits;
-    const float f = std::isinf(inside) ? 4.0f : inside;
     std::memcpy(&bits, &f, 4);
     T.cell_fast[c] = (bits & ~15u) | static_cast<uint32_t>(cnt);
   }
-  // every threshold must be farther than 2^-17 from every cell edge
+  // every midpoint must be farther than 2^-17 from every cell edge
   for (int i = 0; i < 15; ++i) {
-    const double d = std::fabs(thr[i] * 16.0 - std::nearbyint(thr[i] * 16.0)) / 16.0;
+    const double d = std::fabs(mid[i] * 16.0 - std::nearbyint(mid[i] * 16.0)) / 16.0;
     if (d <= std::ldexp(1.0, -17)) T.fast_ok = 0;
   }
   return T;
@@ -628,6 +629,25 @@ void* noalloc_scratch(int dev) {
 }  // namespace
 
 // ======================================================================= ABI
+// Persistent quantizer: one CTA per SM (its shared-memory ring fills most of
+// the SM), never more CTAs than groups.
+template <int kMode>
+int launch_quantize(int64_t groups, int sms, int dev, cudaStream_t st, const float* W, int64_t n_blocks,
+                    uint8_t* codes, uint8_t* q8, float* s2) {
+  auto kern = quantize_nf4_kernel<kMode>;
+  static bool attr_set[kMaxDevices];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(QuantSmem)) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const int64_t grid = std::min<int64_t>(groups, sms);
+  return launch_ex(kern, dim3(static_cast<unsigned>(grid)), dim3(kQuantThreads), sizeof(QuantSmem), st, 1, 1, W,
+                   n_blocks, groups, codes, q8, s2, tables());
+}
+
 extern "C" {
 
 const char* qlora_strerror(int code) {
@@ -662,8 +682,7 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_nf4_kernel<kQuantLinear8>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
-                     1, W, n_blocks, codes, q8, s2, tables());
+    return launch_quantize<kQuantLinear8>(groups, sms, dev, st, W, n_blocks, codes, q8, s2);
   });
 }
 
@@ -680,8 +699,7 @@ int qlora_quantize_nf4_dq_fp8(const float* W, int64_t n_out, int64_t k_in, uint8
   if (groups > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_nf4_kernel<kQuantFp8>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st,
-                     1, 1, W, n_blocks, codes, q8, s2, tables());
+    return launch_quantize<kQuantFp8>(groups, sms, dev, st, W, n_blocks, codes, q8, s2);
   });
 }
 
@@ -698,8 +716,7 @@ int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* cod
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* no_q8 = nullptr;
   return timed(QLORA_KERNEL_QUANTIZE, st, [&] {
-    return launch_ex(quantize_nf4_kernel<kQuantSingle>, dim3(static_cast<unsigned>(groups)), dim3(kQuantThreads), 0, st, 1,
-                     1, W, n_blocks, codes, no_q8, absmax, tables());
+    return launch_quantize<kQuantSingle>(groups, sms, dev, st, W, n_blocks, codes, no_q8, absmax);
   });
 }
 
