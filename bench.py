@@ -42,6 +42,25 @@ CPU_SAMPLE_TOKENS = 4096      # cpu_baseline: tokens of the oracle's sample step
 REF_SAMPLE_TOKENS = 64        # --impl reference: tokens per sampled step
 
 
+class L2Flush:
+    """L2 flush between timed iterations: a write of L2_FLUSH_BYTES, then a
+    read of a second buffer of the same size, so that the lines the write
+    left dirty are written back here rather than inside the next timed
+    kernel (which would otherwise pay for up to an L2's worth of write-back
+    traffic that is not its own)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def __call__(self, i=0):
+        import torch
+        self.w.fill_(float(i))
+        torch.sum(self.r, dim=0, out=self.acc)
+
+
 def step_flops(M, N, K, r):
     """Algorithmic FLOP of fwd + bwd: main 4MNK, LoRA fwd 2Mr(K+N), LoRA bwd 2Mr(N+K) + 2rMK + 2NMr."""
     return 4 * M * N * K + 2 * M * r * (K + N) + 2 * M * r * (N + K) + 2 * r * M * K + 2 * N * M * r
@@ -417,7 +436,7 @@ def run_quant_variant(q, dev, peaks, variant, reps=20):
     gen.manual_seed(3)
     W = gpu_weight(gen, N, K, "normal", dev)
     codes = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     if variant == "single":
         q8 = None
         s2 = torch.empty(N * K // 64, dtype=torch.float32, device=dev)
@@ -430,7 +449,7 @@ def run_quant_variant(q, dev, peaks, variant, reps=20):
         qfn = lambda: q.qlora_quantize_nf4_dq_fp8(W, codes, q8, s2)
 
     def quant():
-        flush.fill_(0.0)
+        flush(0.0)
         qfn()
 
     # time the quantize launches alone: events around each, after an L2 flush
@@ -438,7 +457,7 @@ def run_quant_variant(q, dev, peaks, variant, reps=20):
         quant()
     ev = []
     for _ in range(reps):
-        flush.fill_(0.0)
+        flush(0.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         qfn()
@@ -586,7 +605,7 @@ def run_ours(args, rank, world, local_rank):
     dA = torch.empty(r, K, dtype=torch.float32, device=dev)
     dB = torch.empty(N, r, dtype=torch.float32, device=dev)
     ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
 
     def step(Wd=W, Xd=X, dYd=dY, Ad=A, Bd=B):
         q.qlora_quantize_nf4_dq(Wd, codes, q8, s2)
@@ -601,7 +620,8 @@ def run_ours(args, rank, world, local_rank):
     if args.profile:
         # profiling case for ncu: one step to load the modules, one step to
         # capture, then two decode forwards (M = 1, r = 8) on the same weight.
-        # Launches: [L2 fill + 6 step kernels] x 2, then 2 decode kernels.
+        # Launches: [L2 flush write + L2 flush read + 6 step kernels] x 2, then
+        # 2 decode kernels.
         from bit_nf4_quantized_quantize_b200 import synth
         dinp = synth.layer_inputs("decode", M=1)
         decX, decA, decB = (torch.from_numpy(dinp[k].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -609,7 +629,7 @@ def run_ours(args, rank, world, local_rank):
         decY = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
         dws = torch.empty(q.qlora_workspace_bytes(1, N, K, DECODE_RANK), dtype=torch.uint8, device=dev)
         for i in range(2):
-            flush.fill_(float(i))
+            flush(float(i))
             step()
         for _ in range(2):
             q.qlora_linear_fwd(codes, q8, s2, N, K, decX, decA, decB, dinp["alpha"], Y=decY, workspace=dws)
@@ -621,7 +641,7 @@ def run_ours(args, rank, world, local_rank):
         return
 
     for i in range(args.warmup):
-        flush.fill_(float(i))
+        flush(float(i))
         step()
     torch.cuda.synchronize()
     rc = q.qlora_device_status()
@@ -640,7 +660,7 @@ def run_ours(args, rank, world, local_rank):
     n0 = q.qlora_launch_count()
     t_wall = time.perf_counter()
     for i in range(args.steps):
-        flush.fill_(float(i))          # L2 flush between steps, outside the step's events
+        flush(float(i))          # L2 flush between steps, outside the step's events
         ev[i][0].record()
         step()
         ev[i][1].record()
@@ -662,7 +682,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     q.qlora_timing_enable(True)
     for i in range(args.steps):
-        flush.fill_(float(i))
+        flush(float(i))
         step()
     torch.cuda.synchronize()
     kern = q.qlora_timing_collect()
@@ -683,7 +703,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     for i in range(n_e2e):
-        flush.fill_(float(i))
+        flush(float(i))
         e_ev[i][0].record()
         W.copy_(hW, non_blocking=True)
         X.copy_(hX, non_blocking=True)
@@ -732,7 +752,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": "train4096: one 4096x4096 NF4+DQ layer, M=4096 tokens (4x1024), r=64, alpha=16; "
                                "step = quantize + fwd + bwd",
                    "N": N, "K": K, "M": M, "r": r, "alpha": alpha,
-                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the step events)",
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a {L2_FLUSH_BYTES >> 20} MiB read "
+                         "that writes back the dirty lines; outside the step events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "roofline": roof,
         "quantize": {"gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],

@@ -629,6 +629,36 @@ void* noalloc_scratch(int dev) {
 }  // namespace
 
 // ======================================================================= ABI
+// A second stream per device for backward: the gradient kernel (dA, dB)
+// needs only V, U, X and dY, so it runs beside the dX kernel and takes the
+// SMs that the dX grid's last wave leaves idle.  The library forks it off the
+// caller's stream with an event and joins it back before returning, so the
+// caller sees one ordered stream.  Created on first use, kept for the
+// process's lifetime.
+struct AuxStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+  bool ok = false;
+};
+std::mutex g_aux_mu;
+AuxStream g_aux[kMaxDevices];
+
+// Caller holds g_aux_mu.  nullptr if the stream or events cannot be made.
+AuxStream* aux_stream(int dev) {
+  AuxStream& a = g_aux[dev];
+  if (!a.ok) {
+    if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    a.ok = true;
+  }
+  return &a;
+}
+
 // Persistent quantizer: one CTA per SM (its shared-memory ring fills most of
 // the SM), never more CTAs than groups.
 template <int kMode>
@@ -934,6 +964,19 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev)) return rc;
     U = Ubuf;
   }
+  // The gradient kernel goes to the device's second stream, forked here and
+  // launched after dX so that dX's CTAs are queued first; with per-kernel
+  // timing on, every kernel stays on the caller's stream (each timed alone).
+  std::unique_lock<std::mutex> aux_lk(g_aux_mu, std::defer_lock);
+  AuxStream* aux = nullptr;
+  if (!g_timing_on && dX) {
+    aux_lk.lock();
+    aux = aux_stream(dev);
+    if (aux && cudaEventRecord(aux->fork, st) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+  }
   // dX = dY dequant(W) + (s V) A; with dropout the adapter term is masked, so
   // the fused kernel computes dY dequant(W) alone and dropout_dx_kernel adds
   // s/(1-p) (V A) where the input was kept
@@ -1004,9 +1047,21 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0, 1.f, s);
     la.tiles0 = tiles_a;
     la.r = r;
-    if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, st, dev,
+    cudaStream_t gst = st;
+    if (aux) {
+      if (cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess) {
+        cudaGetLastError();
+        return QLORA_ERR_CUDA;
+      }
+      gst = aux->s;
+    }
+    if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, gst, dev,
                                          QLORA_KERNEL_GRAD_GEMM))
       return rc;
+    if (aux && (cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
   }
   return QLORA_OK;
 }
