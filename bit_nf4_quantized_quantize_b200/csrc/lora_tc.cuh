@@ -25,7 +25,6 @@
 
 namespace qlora {
 
-constexpr int kLoraStages = 4;
 constexpr int kLoraBN = 64;
 constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
@@ -55,35 +54,41 @@ struct LoraArgs {
   int r;
 };
 
+// Shared memory of one CTA: STAGES pipeline stages, each KB reduction steps
+// of 64 (an A tile of 128 x 64 and a B tile of 64 x 64 bf16 per step).
+template <int STAGES, int KB>
 struct LoraSmem {
   static constexpr int kATile = 128 * 64 * 2;   // 16 KiB
   static constexpr int kBTile = 64 * 64 * 2;    // 8 KiB
+  static constexpr int kAStage = KB * kATile;
+  static constexpr int kBStage = KB * kBTile;
   static constexpr int kAOff = 0;
-  static constexpr int kBOff = kAOff + kLoraStages * kATile;
-  static constexpr int kBarOff = kBOff + kLoraStages * kBTile;   // 96 KiB
-  static constexpr int kMiscOff = kBarOff + (2 * kLoraStages + 1) * 8;
+  static constexpr int kBOff = kAOff + STAGES * kAStage;
+  static constexpr int kBarOff = kBOff + STAGES * kBStage;
+  static constexpr int kMiscOff = kBarOff + (2 * STAGES + 1) * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kDynBytes = kBytes + 1024;
   static constexpr int kRedBytes = 128 * 64 * 4;  // fp32 accumulator copy (reuses the A stages)
   static_assert(kRedBytes <= kBOff, "reduction buffer fits in the A stages");
+  static_assert(kDynBytes <= 232448, "shared memory");
 };
 
 // A_MN: A operand MN-major (dA^T = X^T V, dB = dY^T U); else K-major (U, V).
 // B_MN: B operand MN-major (V = dY B and the gradient products); else K-major (U).
-template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kLoraThreads, 2)
+// STAGES pipeline stages of KB reduction steps each.
+template <bool A_MN, bool B_MN, int STAGES, int KB>
+__global__ void __launch_bounds__(kLoraThreads, 1)
 qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                   const LoraArgs args) {
-  using L = LoraSmem;
+  using L = LoraSmem<STAGES, KB>;
   constexpr uint32_t kIdesc = idesc_bf16_m128(kLoraBN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
-  constexpr uint32_t kTxBytes = L::kATile + L::kBTile;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* empty = full + kLoraStages;
-  uint64_t* accum_full = empty + kLoraStages;
+  uint64_t* empty = full + STAGES;
+  uint64_t* accum_full = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -98,10 +103,11 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   const int S = static_cast<int>(gridDim.z);     // cluster size along z
   const int rank = static_cast<int>(cluster_ctarank());
   const int ks0 = rank * P.per_split;
-  const int n_steps = max(0, min(P.k_steps, ks0 + P.per_split) - ks0);
+  const int n_steps = max(0, min(P.k_steps, ks0 + P.per_split) - ks0);   // reduction steps of 64
+  const int n_stages = (n_steps + KB - 1) / KB;                             // pipeline iterations
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kLoraStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -121,37 +127,43 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
     if (lane == 0) {
       tma_prefetch_desc(tA);
       tma_prefetch_desc(tB);
-      for (int t = 0; t < n_steps; ++t) {
-        const int s = t % kLoraStages;
-        if (t >= kLoraStages && !mbar_wait(&empty[s], ((t / kLoraStages) - 1) & 1, abort_flag)) break;
-        const int ks = ks0 + t;
-        uint8_t* a_dst = smem + L::kAOff + s * L::kATile;
-        uint8_t* b_dst = smem + L::kBOff + s * L::kBTile;
-        mbar_arrive_expect_tx(&full[s], kTxBytes);
-        if (A_MN) {
-          tma_load_2d(a_dst, tA, &full[s], m0, ks * 64);
-          tma_load_2d(a_dst + 64 * 128, tA, &full[s], m0 + 64, ks * 64);
-        } else {
-          tma_load_2d(a_dst, tA, &full[s], ks * 64, m0);
+      for (int t = 0; t < n_stages; ++t) {
+        const int s = t % STAGES;
+        if (t >= STAGES && !mbar_wait(&empty[s], ((t / STAGES) - 1) & 1, abort_flag)) break;
+        const int nb = min(KB, n_steps - t * KB);
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nb * (L::kATile + L::kBTile)));
+        for (int b = 0; b < nb; ++b) {
+          const int ks = ks0 + t * KB + b;
+          uint8_t* a_dst = smem + L::kAOff + s * L::kAStage + b * L::kATile;
+          uint8_t* b_dst = smem + L::kBOff + s * L::kBStage + b * L::kBTile;
+          if (A_MN) {
+            tma_load_2d(a_dst, tA, &full[s], m0, ks * 64);
+            tma_load_2d(a_dst + 64 * 128, tA, &full[s], m0 + 64, ks * 64);
+          } else {
+            tma_load_2d(a_dst, tA, &full[s], ks * 64, m0);
+          }
+          if (B_MN) tma_load_2d(b_dst, tB, &full[s], c0, ks * 64);
+          else tma_load_2d(b_dst, tB, &full[s], ks * 64, c0);
         }
-        if (B_MN) tma_load_2d(b_dst, tB, &full[s], c0, ks * 64);
-        else tma_load_2d(b_dst, tB, &full[s], ks * 64, c0);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    for (int t = 0; t < n_steps; ++t) {
-      const int s = t % kLoraStages;
-      if (!mbar_wait(&full[s], (t / kLoraStages) & 1, abort_flag)) break;
+    for (int t = 0; t < n_stages; ++t) {
+      const int s = t % STAGES;
+      if (!mbar_wait(&full[s], (t / STAGES) & 1, abort_flag)) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kATile);
-        const uint32_t b_base = smem_u32(smem + L::kBOff + s * L::kBTile);
+        const int nb = min(KB, n_steps - t * KB);
+        for (int b = 0; b < nb; ++b) {
+          const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kAStage + b * L::kATile);
+          const uint32_t b_base = smem_u32(smem + L::kBOff + s * L::kBStage + b * L::kBTile);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 64 * 128) : smem_desc_sw128(a_base + kk * 32, 16);
-          const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 64 * 128) : smem_desc_sw128(b_base + kk * 32, 16);
-          umma_bf16(tmem_d, ad, bd, kIdesc, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 64 * 128) : smem_desc_sw128(a_base + kk * 32, 16);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 64 * 128) : smem_desc_sw128(b_base + kk * 32, 16);
+            umma_bf16(tmem_d, ad, bd, kIdesc, (t > 0 || b > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -256,7 +268,11 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
     }
   }
 
-  cluster_sync_all();   // no rank leaves while another still reads its shared memory
+  // No rank leaves while another still reads its shared memory.  Every remote
+  // value was consumed before this point, so a relaxed arrive suffices and
+  // the barrier does not wait for this CTA's global stores to complete.
+  cluster_arrive_relaxed();
+  cluster_wait();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_d, kLoraBN);

@@ -464,13 +464,18 @@ int gemm_split(int tiles, int k_steps, int dev) {
                         64 + 32 * 8, L::kDynBytes, tiles, k_steps, 2, false, dev);
 }
 
-template <bool A_MN, bool B_MN>
+// Pipeline shape of the adapter kernel: stages x reduction steps per stage.
+constexpr int kLoraStagesDefault = 4;
+constexpr int kLoraKbDefault = 1;
+
+template <bool A_MN, bool B_MN, int STAGES = kLoraStagesDefault, int KB = kLoraKbDefault>
 int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
                 const LoraArgs& args, int tiles_total, int S, cudaStream_t st, int dev, int kind) {
-  auto kern = qlora_lora_kernel<A_MN, B_MN>;
+  auto kern = qlora_lora_kernel<A_MN, B_MN, STAGES, KB>;
+  using L = LoraSmem<STAGES, KB>;
   static bool attr_set[kMaxDevices];
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LoraSmem::kDynBytes) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
       cudaGetLastError();
       return QLORA_ERR_CUDA;
     }
@@ -478,7 +483,7 @@ int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap&
   }
   return timed(kind, st, [&] {
     return launch_ex(kern, dim3(static_cast<unsigned>(tiles_total), 1, static_cast<unsigned>(S)), dim3(kLoraThreads),
-                     LoraSmem::kDynBytes, st, 1, static_cast<unsigned>(S), a0, b0, a1, b1, args);
+                     L::kDynBytes, st, 1, static_cast<unsigned>(S), a0, b0, a1, b1, args);
   });
 }
 
