@@ -107,12 +107,22 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-def kernel_source_hash():
+# Device sources of each timed kernel kind (csrc/): a capture's DRAM traffic
+# stays valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "fwd_fused": ("fused2_tc.cuh", "gemm_tc.cuh", "ptx_sm100.cuh"),
+    "dx_fused": ("fused2_tc.cuh", "gemm_tc.cuh", "ptx_sm100.cuh"),
+    "quantize": ("quantize.cuh", "ptx_sm100.cuh"),
+    "lora_gemm": ("lora_tc.cuh", "ptx_sm100.cuh"),
+    "grad_gemm": ("lora_tc.cuh", "ptx_sm100.cuh"),
+}
+
+
+def kernel_source_hash(kind):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_nf4_quantized_quantize_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kind]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -123,7 +133,7 @@ def load_traffic(kind):
         return None
     d = json.load(open(p))
     e = d.get(kind)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or kind not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kind):
         return None
     return e.get("bytes_per_launch")
 
