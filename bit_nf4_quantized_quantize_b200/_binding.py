@@ -251,7 +251,13 @@ def qlora_workspace_bytes(M: int, n_out: int, k_in: int, r: int) -> int:
     return int(load().qlora_workspace_bytes(M, n_out, k_in, r))
 
 
+def _nbytes(ws):
+    return 0 if ws is None else ws.numel()
+
+
 def _workspace(ws, M, N, K, r, device):
+    if M == 0:
+        return ws   # an empty batch needs no workspace
     need = qlora_workspace_bytes(M, N, K, r)
     if need == 0:
         raise QloraError(-2, "qlora_workspace_bytes")
@@ -274,7 +280,7 @@ def qlora_linear_fwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float
         _dev(U_save, torch.bfloat16, "U_save", (M, r))
     ws = _workspace(workspace, M, n_out, k_in, r, X.device)
     _check(load().qlora_linear_fwd(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A), _ptr(B), r,
-                                   float(alpha), _ptr(Y), _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)),
+                                   float(alpha), _ptr(Y), _ptr(U_save), _ptr(ws), _nbytes(ws), _stream(stream)),
            "qlora_linear_fwd")
     return Y
 
@@ -320,7 +326,7 @@ def qlora_linear_bwd(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float
     ws = _workspace(workspace, M, n_out, k_in, r, dev)
     _check(load().qlora_linear_bwd(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A), _ptr(B), r,
                                    float(alpha), _ptr(dY), _ptr(U_saved), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
-                                   ws.numel(), _stream(stream)),
+                                   _nbytes(ws), _stream(stream)),
            "qlora_linear_bwd")
     return dX, dA, dB
 
@@ -330,6 +336,8 @@ def qlora_workspace_bytes_dropout(M: int, n_out: int, k_in: int, r: int) -> int:
 
 
 def _workspace_dropout(ws, M, N, K, r, device):
+    if M == 0:
+        return ws   # an empty batch needs no workspace
     need = qlora_workspace_bytes_dropout(M, N, K, r)
     if need == 0:
         raise QloraError(-2, "qlora_workspace_bytes_dropout")
@@ -353,7 +361,7 @@ def qlora_linear_fwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
     ws = _workspace_dropout(workspace, M, n_out, k_in, r, X.device)
     _check(load().qlora_linear_fwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
                                            _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(Y),
-                                           _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)),
+                                           _ptr(U_save), _ptr(ws), _nbytes(ws), _stream(stream)),
            "qlora_linear_fwd_dropout")
     return Y
 
@@ -381,7 +389,7 @@ def qlora_linear_bwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
     ws = _workspace_dropout(workspace, M, n_out, k_in, r, dev)
     _check(load().qlora_linear_bwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
                                            _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(dY),
-                                           _ptr(U_saved), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                                           _ptr(U_saved), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), _nbytes(ws),
                                            _stream(stream)),
            "qlora_linear_bwd_dropout")
     return dX, dA, dB

@@ -514,12 +514,22 @@ int check_weight(const uint8_t* codes, const uint8_t* q8, const float* s2, int64
   return QLORA_OK;
 }
 
+// M == 0 (an empty batch) is valid, and X may then be NULL.
 int check_lora(const void* X, int64_t M, const void* A, const void* B, int r, float alpha) {
-  if (!X || !A || !B) return QLORA_ERR_INVALID_ARG;
-  if (M < 1 || M > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if ((M != 0 && !X) || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (M < 0 || M > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
   if (r % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if ((X && !aligned16(X)) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+// Shape of a weight for the quantizer, the dequantizer and the merge: n_out,
+// k_in >= 0 with k_in % 64 == 0.  Sets *empty when it holds no element (the
+// call is then a no-op and its pointers may be NULL).
+int check_weight_shape(int64_t n_out, int64_t k_in, bool* empty) {
+  if (n_out < 0 || k_in < 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  *empty = n_out == 0 || k_in == 0;
   return QLORA_OK;
 }
 
@@ -706,8 +716,10 @@ int qlora_nf4_codebook(float* out) {
 
 int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, uint8_t* q8, float* s2,
                           void* stream) {
+  bool empty;
+  if (int rc = check_weight_shape(n_out, k_in, &empty)) return rc;
+  if (empty) return QLORA_OK;
   if (!W || !codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
-  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(s2) & 3u))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
@@ -723,8 +735,10 @@ int qlora_quantize_nf4_dq(const float* W, int64_t n_out, int64_t k_in, uint8_t* 
 
 int qlora_quantize_nf4_dq_fp8(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, uint8_t* q8, float* s2,
                               void* stream) {
+  bool empty;
+  if (int rc = check_weight_shape(n_out, k_in, &empty)) return rc;
+  if (empty) return QLORA_OK;
   if (!W || !codes || !q8 || !s2) return QLORA_ERR_INVALID_ARG;
-  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(s2) & 3u))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
@@ -739,8 +753,10 @@ int qlora_quantize_nf4_dq_fp8(const float* W, int64_t n_out, int64_t k_in, uint8
 }
 
 int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* codes, float* absmax, void* stream) {
+  bool empty;
+  if (int rc = check_weight_shape(n_out, k_in, &empty)) return rc;
+  if (empty) return QLORA_OK;
   if (!W || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
-  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(absmax) & 3u))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
@@ -757,11 +773,13 @@ int qlora_quantize_nf4(const float* W, int64_t n_out, int64_t k_in, uint8_t* cod
 
 int qlora_merge_adapter(const float* W, int64_t n_out, int64_t k_in, const uint16_t* A, const uint16_t* B, int r,
                         float alpha, void* out, int out_dtype, void* stream) {
-  if (!W || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
   if (out_dtype != QLORA_OUT_BF16 && out_dtype != QLORA_OUT_FP32) return QLORA_ERR_INVALID_ARG;
   if (r < 1 || r > 256 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0 || n_out > (1 << 24) || k_in > (1 << 24))
-    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  bool empty;
+  if (int rc = check_weight_shape(n_out, k_in, &empty)) return rc;
+  if (n_out > (1 << 24) || k_in > (1 << 24)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (empty) return QLORA_OK;
+  if (!W || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
@@ -782,9 +800,11 @@ int qlora_merge_adapter(const float* W, int64_t n_out, int64_t k_in, const uint1
 
 int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
                   void* out, int out_dtype, void* stream) {
-  if (!codes || !s2 || !out) return QLORA_ERR_INVALID_ARG;   // q8 == NULL: single quantization
   if (out_dtype != QLORA_OUT_BF16 && out_dtype != QLORA_OUT_FP32) return QLORA_ERR_INVALID_ARG;
-  if (n_out <= 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  bool empty;
+  if (int rc = check_weight_shape(n_out, k_in, &empty)) return rc;
+  if (empty) return QLORA_OK;
+  if (!codes || !s2 || !out) return QLORA_ERR_INVALID_ARG;   // q8 == NULL: single quantization
   if ((reinterpret_cast<uintptr_t>(codes) & 3u) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
@@ -801,7 +821,7 @@ int qlora_dequant(const uint8_t* codes, const uint8_t* q8, const float* s2, int6
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r) {
-  if (M < 1 || n_out < 64 || k_in < 64 || r < 1 || r > 256) return 0;
+  if (M < 1 || n_out < 64 || k_in < 64 || r < 1 || r > 256) return 0;   // M == 0 needs no workspace
   int dev = 0, sms = 148;
   if (check_device(&dev, &sms) != QLORA_OK) sms = 148;
   return ws_layout(M, n_out, k_in, r, sms).total;
@@ -814,6 +834,7 @@ static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
                     const DropoutSpec& dr) {
   if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
   if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
+  if (M == 0) return QLORA_OK;   // an empty batch: Y and U have no rows
   if (!Y) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
@@ -906,6 +927,7 @@ int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const floa
                              int r, float alpha, uint16_t* Y, uint16_t* U_save, void* stream) {
   if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
   if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
+  if (M == 0) return QLORA_OK;   // an empty batch: nothing to compute
   if (!Y) return QLORA_ERR_INVALID_ARG;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
@@ -924,12 +946,22 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
                     void* workspace, size_t workspace_bytes, void* stream, const DropoutSpec& dr) {
   if (int rc = check_weight(codes, q8, s2, n_out, k_in)) return rc;
   if (int rc = check_lora(X, M, A, B, r, alpha)) return rc;
-  if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (U_saved && !aligned16(U_saved)) ||
+  if ((M != 0 && !dY) || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if ((dY && !aligned16(dY)) || !aligned16(dA) || !aligned16(dB) || (U_saved && !aligned16(U_saved)) ||
       (dX && !aligned16(dX)))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
+  if (M == 0) {
+    // an empty batch: the sums over tokens that make dA and dB are empty, so both are zero
+    cudaStream_t st0 = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(dA, 0, sizeof(float) * static_cast<size_t>(r) * static_cast<size_t>(k_in), st0) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, sizeof(float) * static_cast<size_t>(n_out) * static_cast<size_t>(r), st0) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+  }
   const WsLayout L = ws_layout(M, n_out, k_in, r, sms, dr.on);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QLORA_ERR_WORKSPACE;
@@ -1099,11 +1131,12 @@ size_t qlora_workspace_bytes_dropout(int64_t M, int64_t n_out, int64_t k_in, int
 
 int qlora_dropout_apply(const uint16_t* X, int64_t M, int64_t k_in, float p, uint64_t seed, uint64_t offset,
                         uint16_t* out, void* stream) {
-  if (!X || !out) return QLORA_ERR_INVALID_ARG;
-  if (M < 1 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(X) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M < 0 || k_in <= 0 || k_in % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
   DropoutSpec dr;
   if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;   // an empty batch
+  if (!X || !out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(out)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;
   if (int rc = check_device(&dev, &sms)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -40,8 +40,16 @@
  *   quantization.  Fixed by the method: block 64, group 256.
  * - Preconditions checked on the host (QLORA_ERR_* on violation, nothing
  *   enqueued): non-NULL required pointers, every pointer 16-byte aligned,
- *   K % 64 == 0, N % 64 == 0, M >= 1, 1 <= r <= 256 with r % 8 == 0, alpha
- *   finite.  NaN or Inf inside W is a caller error; the result is unspecified.
+ *   K % 64 == 0, N % 64 == 0 (N, K >= 64 for the layer), M >= 0,
+ *   1 <= r <= 256 with r % 8 == 0, alpha finite.  NaN or Inf inside W is a
+ *   caller error; the result is unspecified.
+ * - Empty inputs.  M == 0 (an empty batch, e.g. a data-parallel rank that
+ *   received no tokens) is valid: the forward enqueues nothing, the backward
+ *   sets dA and dB to zero (sums over no tokens) and nothing else, and the
+ *   pointers to M-row buffers (X, Y, U, dY, dX) may be NULL.  A weight with
+ *   no element (n_out == 0 or k_in == 0) makes the quantizers, the
+ *   dequantizer and the merge no-ops whose pointers may be NULL.  The layer
+ *   itself needs N, K >= 64.
  * - Return value: QLORA_OK (0) or a negative QLORA_ERR_* code.  Errors raised
  *   on the device after a call returned (a bounded wait inside a kernel that
  *   gave up) are latched in a device flag and reported by qlora_device_status.

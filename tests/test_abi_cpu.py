@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import bit_nf4_quantized_quantize_b200 as q
@@ -84,15 +85,18 @@ def test_host_validation_without_gpu(lib):
     assert fwd(Y=0) == -1
     assert fwd(K=100) == -2
     assert fwd(N=100) == -2
-    assert fwd(M=0) == -2
+    assert fwd(M=-1) == -2
+    # an empty batch is valid without any buffer or workspace, and touches no device
+    assert fwd(M=0, X=0, Y=0, ws=0, wsb=0) == 0
     assert fwd(r=0) == -1
     assert fwd(r=300) == -1
     assert fwd(r=12) == -2
     assert fwd(alpha=float("nan")) == -1
     assert fwd(X=P + 8) == -2
-    # everything valid: the first CUDA query fails on a machine without a B200
-    rc = fwd()
-    assert rc in (-6, -5, 0) or rc == -3
+    # everything valid: the first CUDA query fails on a machine without a B200.  (With a GPU
+    # visible this call would launch kernels on the fake addresses, so it runs only without one.)
+    if not torch.cuda.is_available():
+        assert fwd() in (-6, -3)
 
     def bwd(dY=P, dA=P, dB=P):
         return lib.qlora_linear_bwd(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
@@ -103,6 +107,11 @@ def test_host_validation_without_gpu(lib):
     assert bwd(dA=0) == -1
     assert bwd(dB=0) == -1
     assert bwd(dY=P + 2) == -2
+    # an empty weight: the quantizers and the dequantizer are no-ops on NULL buffers
+    assert lib.qlora_quantize_nf4_dq(null, 0, 64, null, null, null, null) == 0
+    assert lib.qlora_quantize_nf4(null, 64, 0, null, null, null) == 0
+    assert lib.qlora_dequant(null, null, null, 0, 64, null, 0, null) == 0
+    assert lib.qlora_quantize_nf4_dq(null, -1, 64, null, null, null, null) == -2
 
 
 def test_binding_refuses_cpu_tensors(lib):

@@ -169,3 +169,34 @@ def test_fp8_second_stage_linear(M, N, K, r):
     """The layer on a weight whose second stage is FP8-E4M3 (sign-tagged s2):
     forward and backward against the oracle."""
     run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=800 + M), fp8=True)
+
+
+def test_empty_batch_and_empty_weight():
+    """M = 0: the forward writes nothing; the backward's dA and dB are sums over no tokens, so
+    both are zero, as the oracle gives (prefilled NaN must be overwritten).  A weight with no
+    element quantizes and dequantizes to empty buffers."""
+    inp = synth.layer_inputs("tiny")
+    N, K, r, alpha = inp["N"], inp["K"], inp["r"], inp["alpha"]
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    A, B = to_dev_bf16(inp["A"]), to_dev_bf16(inp["B"])
+    X = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    dY = torch.empty(0, N, dtype=torch.bfloat16, device="cuda")
+    Y = q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha)
+    assert tuple(Y.shape) == (0, N)
+    dA = torch.full((r, K), float("nan"), device="cuda")
+    dB = torch.full((N, r), float("nan"), device="cuda")
+    dX, dA, dB = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert q.qlora_device_status() == 0
+    What = oracle_weight(inp["W"])[3]
+    _, dAr, dBr = oracle.linear_bwd(np.zeros((0, K)), What, bits_f64(inp["A"]), bits_f64(inp["B"]),
+                                    np.zeros((0, N)), alpha)
+    assert tuple(dX.shape) == (0, K)
+    assert np.array_equal(dA.cpu().numpy(), dAr) and np.array_equal(dB.cpu().numpy(), dBr)
+    assert not dAr.any() and not dBr.any()
+    # empty weight: no-op quantize and dequantize
+    for shape in ((0, 256), (64, 0)):
+        c, qq, ss = q.qlora_quantize_nf4_dq(torch.empty(*shape, device="cuda"))
+        assert c.numel() == 0 and qq.numel() == 0 and ss.numel() == 0
+        assert q.qlora_dequant(c, qq, ss, *shape).numel() == 0
+    assert q.qlora_device_status() == 0
