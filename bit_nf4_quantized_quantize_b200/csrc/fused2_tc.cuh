@@ -180,7 +180,11 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   cluster_barrier();     // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
-  griddep_wait();   // no global access before the previous grid is complete
+  // The previous grid on the stream is the adapter kernel that writes s U
+  // (or s V); it releases this grid as soon as it is running.  The main steps
+  // read only X (or dY) and the packed weight, which are complete before that
+  // kernel started, so the wait for its completion comes just before the
+  // first adapter slice (producer) and before the first store (epilogue).
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (each CTA its own halves)
@@ -193,19 +197,21 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         if (t >= NST && !mbar_wait(&empty[s], ((t / NST) - 1) & 1, abort_flag)) break;
         uint8_t* a_dst = smem + L::kAOff + s * L::kATile;
         uint8_t* b_dst = smem + L::kBOff + s * L::kBTile;
-        if (t < n_lora) {
+        if (t >= n_main) {
+          const int j = t - n_main;   // adapter slice: the previous grid's output
+          if (j == 0) griddep_wait();
           mbar_arrive_expect_tx(&full_tma[s], L::kATile + L::kBTile);
 #pragma unroll
           for (int h = 0; h < MH; ++h)
-            tma_load_2d(a_dst + h * kAHalfBytes, &tmA2, &full_tma[s], t * kBK, m0 + 256 * h + 128 * rank);
+            tma_load_2d(a_dst + h * kAHalfBytes, &tmA2, &full_tma[s], j * kBK, m0 + 256 * h + 128 * rank);
           if (!kBMN) {
-            tma_load_2d(b_dst, &tmB2, &full_tma[s], t * kBK, cb);
+            tma_load_2d(b_dst, &tmB2, &full_tma[s], j * kBK, cb);
           } else {
-            tma_load_2d(b_dst, &tmB2, &full_tma[s], cb, t * kBK);
-            tma_load_2d(b_dst + kBK * 128, &tmB2, &full_tma[s], cb + 64, t * kBK);
+            tma_load_2d(b_dst, &tmB2, &full_tma[s], cb, j * kBK);
+            tma_load_2d(b_dst + kBK * 128, &tmB2, &full_tma[s], cb + 64, j * kBK);
           }
         } else {
-          const int ks = t - n_lora;
+          const int ks = t;
           mbar_arrive_expect_tx(&full_tma[s], L::kATile + L::kPTile);
 #pragma unroll
           for (int h = 0; h < MH; ++h)
@@ -260,16 +266,15 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const int64_t blk = static_cast<int64_t>(wr) * args.w_kblocks + kb;
       return block_scale(args.q8, args.s2, blk);
     };
-    // this warpgroup's main steps are ks = first, first+2, ...; prefetch two ahead
-    const int first = (n_lora + wg) & 1;   // smallest ks with (n_lora + ks) % 2 == wg
-    float c1_a = (first < n_main) ? load_scale(first) : 0.f;
-    float c1_b = (first + 2 < n_main) ? load_scale(first + 2) : 0.f;
+    // this warpgroup's main steps are ks = t = wg, wg+2, ...; scales prefetched two ahead
+    float c1_a = (wg < n_main) ? load_scale(wg) : 0.f;
+    float c1_b = (wg + 2 < n_main) ? load_scale(wg + 2) : 0.f;
     for (int t = wg; t < total; t += 2) {
       const int s = t % NST;
       const uint32_t ph = (t / NST) & 1;
       if (!mbar_wait(&full_tma[s], ph, abort_flag)) { ok = false; break; }
-      if (t >= n_lora) {
-        const int ks = t - n_lora;
+      if (t < n_main) {
+        const int ks = t;
         const float c1 = c1_a;
         c1_a = c1_b;
         if (ks + 4 < n_main) c1_b = load_scale(ks + 4);
@@ -312,6 +317,7 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
     // ------------------------------------------------------------ epilogue (own 128 rows per half)
     if (ok) ok = mbar_wait_cluster(accum_full, 0, abort_flag);
+    griddep_wait();   // the previous grid is complete before this grid writes anything
     griddep_launch_dependents();
     if (ok) {
       tc_fence_after();

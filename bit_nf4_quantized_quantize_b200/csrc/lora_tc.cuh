@@ -100,10 +100,16 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   const int tile = static_cast<int>(blockIdx.x) - (which ? args.tiles0 : 0);
   const int m0 = (tile / P.tiles_n) * 128;
   const int c0 = (tile % P.tiles_n) * kLoraBN;
-  const int S = static_cast<int>(gridDim.z);     // cluster size along z
-  const int rank = static_cast<int>(cluster_ctarank());
+  // The cluster is cx x 1 x S CTAs: the S ranks along z split the reduction;
+  // cx = 2 only places two neighbouring tiles on one TPC (S = 1 then).  The
+  // peer with split rank p has cluster rank x_local + cx * p.
+  const int S = static_cast<int>(gridDim.z);
+  const int rank = static_cast<int>(blockIdx.z);
+  const uint32_t cx = cluster_dim_x();
+  const uint32_t x_local = cluster_ctarank() % cx;
   const int ks0 = rank * P.per_split;
-  const int n_steps = max(0, min(P.k_steps, ks0 + P.per_split) - ks0);   // reduction steps of 64
+  const bool live = tile < P.tiles_m * P.tiles_n;   // false: a CTA that only pads the grid to the cluster
+  const int n_steps = live ? max(0, min(P.k_steps, ks0 + P.per_split) - ks0) : 0;   // reduction steps of 64
   const int n_stages = (n_steps + KB - 1) / KB;                             // pipeline iterations
 
   if (threadIdx.x == 0) {
@@ -121,6 +127,11 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   griddep_wait();   // no global access before the previous grid is complete
+  // Release the next grid now: every CTA of this one is running, so a next
+  // grid that waits for this one's completion (griddep_wait) before reading
+  // its outputs cannot starve it of SMs, and it can start work that does not
+  // depend on them on the SMs this grid leaves free.
+  griddep_launch_dependents();
 
   bool ok = true;
   if (warp == 0) {
@@ -174,7 +185,6 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   } else {
     // copy the accumulator (or zeros, for a rank with no steps) to shared memory
     ok = mbar_wait(accum_full, 0, abort_flag);
-    griddep_launch_dependents();
     float* red = reinterpret_cast<float*>(smem + L::kAOff);
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -205,7 +215,7 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
   __syncthreads();
   cluster_sync_all();   // every rank's accumulator is in its shared memory
 
-  if (warp >= 2 && !*abort_flag) {
+  if (warp >= 2 && live && !*abort_flag) {
     // rows [rank*128/S, (rank+1)*128/S) of the tile, summed over ranks 0..S-1
     const int t = threadIdx.x - 64;            // 0..127
     const int rows_here = 128 / S;
@@ -226,7 +236,7 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
       float4 v[8];
 #pragma unroll
       for (int p = 0; p < 8; ++p)
-        if (p < S) v[p] = ld_cluster_v4(map_to_rank(red_base + off, p));
+        if (p < S) v[p] = ld_cluster_v4(map_to_rank(red_base + off, x_local + cx * static_cast<uint32_t>(p)));
       float4 acc = v[0];
 #pragma unroll
       for (int p = 1; p < 8; ++p)

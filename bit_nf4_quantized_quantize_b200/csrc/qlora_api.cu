@@ -468,9 +468,11 @@ int gemm_split(int tiles, int k_steps, int dev) {
 constexpr int kLoraStagesDefault = 4;
 constexpr int kLoraKbDefault = 1;
 
+// Grid: tiles_total CTAs along x (rounded up to cx) times S along z, in
+// clusters of cx x 1 x S.
 template <bool A_MN, bool B_MN, int STAGES = kLoraStagesDefault, int KB = kLoraKbDefault>
 int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
-                const LoraArgs& args, int tiles_total, int S, cudaStream_t st, int dev, int kind) {
+                const LoraArgs& args, int tiles_total, int S, cudaStream_t st, int dev, int kind, int cx = 1) {
   auto kern = qlora_lora_kernel<A_MN, B_MN, STAGES, KB>;
   using L = LoraSmem<STAGES, KB>;
   static bool attr_set[kMaxDevices];
@@ -482,8 +484,9 @@ int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap&
     attr_set[dev] = true;
   }
   return timed(kind, st, [&] {
-    return launch_ex(kern, dim3(static_cast<unsigned>(tiles_total), 1, static_cast<unsigned>(S)), dim3(kLoraThreads),
-                     L::kDynBytes, st, 1, static_cast<unsigned>(S), a0, b0, a1, b1, args);
+    const unsigned gx = static_cast<unsigned>((tiles_total + cx - 1) / cx * cx);
+    return launch_ex(kern, dim3(gx, 1, static_cast<unsigned>(S)), dim3(kLoraThreads), L::kDynBytes, st,
+                     static_cast<unsigned>(cx), static_cast<unsigned>(S), a0, b0, a1, b1, args);
   });
 }
 
@@ -537,22 +540,45 @@ void fill_levels(GemmArgs& g) {
   for (int i = 0; i < 16; ++i) g.level[i] = tables().level[i];
 }
 
+// V runs beside dX as U runs beside the forward's fused kernel; dX's empty
+// slots also take the gradient kernel (second stream).
+constexpr bool kVBesideDx = true;
+
+// Whether an adapter product (U = X A^T or V = dY B: ceil(M/128) x rpad/64
+// tiles) can run beside the fused kernel that consumes it (`pairs` CTA-pair
+// tiles over the same reduction length).  It then runs unsplit, one CTA per
+// tile, two neighbouring tiles per TPC (a cluster of 2 along x): each of its
+// C clusters takes one CTA-pair slot from the fused kernel's first wave for
+// less than one of that kernel's tiles (one tile is twice the reduction
+// steps at half the rate).  That costs nothing when C does not exceed the
+// pair slots the fused kernel's last wave leaves empty.
+bool adapter_beside(int64_t M, int rpad, int pairs, int num_sms) {
+  if (num_sms < 2) return false;
+  const int64_t tiles = (M + 127) / 128 * (rpad / 64);
+  const int64_t clusters = (tiles + 1) / 2;
+  const int64_t slots = num_sms / 2;
+  const int64_t waves = (pairs + slots - 1) / slots;
+  return clusters <= waves * slots - pairs;
+}
+
 // acc = X A^T; `plain` = bf16(scale0 acc) and `scaled` = bf16(scale1 acc), each may be NULL.
+// beside: the unsplit grid of adapter_beside.
 int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat, int r, float scale0, float scale1,
-                  uint16_t* plain, uint16_t* scaled, int num_sms, cudaStream_t st, int dev) {
+                  uint16_t* plain, uint16_t* scaled, int num_sms, cudaStream_t st, int dev, bool beside = false) {
   const int rpad = (r + 63) / 64 * 64;
   CUtensorMap ta, tb;
   if (!map_bf16(&ta, X, M, K, 64, 128) || !map_bf16(&tb, Amat, r, K, 64, 64)) return QLORA_ERR_CUDA;
   const int k_steps = static_cast<int>(K / 64);
   const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
-  const int S = lora_cluster(tiles, k_steps, num_sms);
+  const int S = beside ? 1 : lora_cluster(tiles, k_steps, num_sms);
   LoraArgs la{};
   la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, plain, scaled, 0, scale0,
                          scale1);
   la.p[1] = la.p[0];
+  la.p[1].tiles_m = 0;   // no second problem: a CTA padding the grid has no tile
   la.tiles0 = tiles;
   la.r = r;
-  return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM);
+  return launch_lora<false, false>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM, beside ? 2 : 1);
 }
 
 // ------------------------------------------------------------------ LoRA dropout
@@ -852,12 +878,16 @@ static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   if (M <= kDecMaxTokens && r <= kDecMaxRank && !dr.on)
     return run_decode(codes, q8, s2, n_out, k_in, X, M, A, B, r, s, Y, U_save, st, dev);
 
+  // the pair path's tiles, and whether U can run beside the fused kernel
+  const int mh = M > 256 ? 2 : 1;
+  const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * static_cast<int>((n_out + 255) / 256);
+  const bool beside = M > 128 && adapter_beside(M, rpad, pairs, sms);
   if (dr.on) {
     // the adapter's input goes through dropout: U = (X * keep) A^T / (1 - p)
     uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
     if (int rc = launch_dropout_mask(X, M, k_in, dr, Xm, sms, st)) return rc;
-    if (int rc = run_lora_down(Xm, M, k_in, A, r, dr.inv, s * dr.inv, U_save, Us, sms, st, dev)) return rc;
-  } else if (int rc = run_lora_down(X, M, k_in, A, r, 1.f, s, U_save, Us, sms, st, dev)) {
+    if (int rc = run_lora_down(Xm, M, k_in, A, r, dr.inv, s * dr.inv, U_save, Us, sms, st, dev, beside)) return rc;
+  } else if (int rc = run_lora_down(X, M, k_in, A, r, 1.f, s, U_save, Us, sms, st, dev, beside)) {
     return rc;
   }
 
@@ -877,14 +907,12 @@ static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   g.split_stride = 0;
   if (M > 128) {
     // CTA pairs: tile (256*MH) x 256, each CTA expanding 128 weight rows per step
-    const int mh = M > 256 ? 2 : 1;
     CUtensorMap tx, tp, tus, tb;
     if (!map_bf16(&tx, X, M, k_in, 64, 128) ||
         !make_map(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k_in / 2, n_out, k_in / 2, 32, 128,
                   CU_TENSOR_MAP_SWIZZLE_32B) ||
         !map_bf16(&tus, Us, M, r, 64, 128) || !map_bf16(&tb, B, n_out, r, 64, 128))
       return QLORA_ERR_CUDA;
-    const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * static_cast<int>((n_out + 255) / 256);
     return mh == 2 ? launch_pair<kBDeqK, 2>(pairs, tx, tp, tus, tb, g, st, dev)
                    : launch_pair<kBDeqK, 1>(pairs, tx, tp, tus, tb, g, st, dev);
   }
@@ -980,13 +1008,22 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     if (!map_bf16(&ta, dY, M, N, 64, 128) || !map_bf16(&tb, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
     const int k_steps = N / 64;
     const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
-    const int S = lora_cluster(tiles, k_steps, sms);
+    // The grid depends on the shapes alone, so V (and with it dA) is the same
+    // bit for bit whichever outputs are requested; it runs beside dX when V is
+    // dX's direct predecessor (U saved, no dropout kernel between).
+    const int mh = M > 256 ? 2 : 1;
+    const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * ((K + 255) / 256);
+    const bool beside = kVBesideDx && M > 128 && adapter_beside(M, rpad, pairs, sms);
+    const int S = beside ? 1 : lora_cluster(tiles, k_steps, sms);
     LoraArgs la{};
     la.p[0] = lora_problem(static_cast<int>(M), k_steps, S, rpad, kLoraOutPlainScaled, V, Vs, 0, 1.f, s);
     la.p[1] = la.p[0];
+    la.p[1].tiles_m = 0;   // no second problem: a CTA padding the grid has no tile
     la.tiles0 = tiles;
     la.r = r;
-    if (int rc = launch_lora<false, true>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM)) return rc;
+    if (int rc = launch_lora<false, true>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM,
+                                          beside ? 2 : 1))
+      return rc;
   }
   // the adapter's input: X, or X * keep with dropout (the 1/(1-p) goes into the scales)
   const uint16_t* Xa = X;
@@ -998,7 +1035,11 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   // U (from the forward, or recomputed)
   const uint16_t* U = U_saved;
   if (!U) {
-    if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev)) return rc;
+    // the forward's grid for U (split or not), so the recomputed U is bit-identical to a saved one
+    const int fmh = M > 256 ? 2 : 1;
+    const int fwd_pairs = static_cast<int>((M + 256 * fmh - 1) / (256 * fmh)) * ((N + 255) / 256);
+    const bool fwd_beside = M > 128 && adapter_beside(M, rpad, fwd_pairs, sms);
+    if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev, fwd_beside)) return rc;
     U = Ubuf;
   }
   // The gradient kernel goes to the device's second stream, forked here and
