@@ -1119,7 +1119,13 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     const int k_steps = static_cast<int>((M + 63) / 64);
     const int tiles_a = ((K + 127) / 128) * (rpad / 64);
     const int tiles_b = ((N + 127) / 128) * (rpad / 64);
-    const int S = lora_cluster(tiles_a + tiles_b, k_steps, sms);
+    // With dX on the CTA-pair path the gradient kernel runs beside it (second
+    // stream) in the slots of dX's last wave: unsplit there, two tiles per TPC,
+    // it takes fewer SM-microseconds than split (train4096 step 238.0 -> 232.0
+    // us) although it is slower alone.  The grid depends on the shapes alone,
+    // so dA and dB have the same bits with or without dX.
+    const bool unsplit = M > 128;
+    const int S = unsplit ? 1 : lora_cluster(tiles_a + tiles_b, k_steps, sms);
     LoraArgs la{};
     la.p[0] = lora_problem(K, k_steps, S, rpad, kLoraOutTransposed, dA, nullptr, K, 1.f, s * dr.inv);
     la.p[1] = lora_problem(N, k_steps, S, rpad, kLoraOutRowMajor, dB, nullptr, 0, 1.f, s);
@@ -1134,7 +1140,7 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
       gst = aux->s;
     }
     if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, gst, dev,
-                                         QLORA_KERNEL_GRAD_GEMM))
+                                         QLORA_KERNEL_GRAD_GEMM, unsplit ? 2 : 1))
       return rc;
     if (aux && (cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)) {
       cudaGetLastError();
