@@ -5,8 +5,8 @@ identical to the GPU's), dequantizes to bf16 and evaluates the layer in fp64 on
 the exact bf16 operands.  Tolerance: relative L2 <= 4e-3 on every output and
 gradient.  Cases span several tiles with ragged tails in M, N and K, adapter
 ranks from 8 to 256 (one to four adapter slices), the tiny and decode
-workloads in full, and the 4096^3 training workload on sampled rows (dA, dB in
-full).
+workloads in full, and the 4096^3 training workload, the 7B down projection and
+the 65B 22016 x 8192 linear on sampled rows (dA, dB in full).
 """
 import numpy as np
 import pytest
@@ -92,6 +92,14 @@ def test_llama7b_down_proj_sampled_rows():
     """The 7B stack's down projection (4096 x 11008, outlier weights), M = 2048."""
     inp = synth.layer_inputs("llama7b", layer=6)
     rows = np.arange(0, 2048, 97)
+    run_case(inp, rows=rows)
+
+
+def test_llama65b_ffn_sampled_rows():
+    """The 65B config's 22016 x 8192 linear (Student-t weights), M = 8192, r = 64, at full size
+    in the bench's launch configuration: Y, U and dX on 32 sampled rows, dA and dB in full."""
+    inp = synth.layer_inputs("llama65b", layer=1)
+    rows = np.unique(np.concatenate([np.arange(0, 8192, 263), [8191]]))
     run_case(inp, rows=rows)
 
 
