@@ -13,8 +13,10 @@
 // The masks are applied where the adapter consumes x:
 //   dropout_mask_kernel   X_keep = X * keep (bf16, exact), the input of U = X_keep A^T
 //                         and dA = V^T X_keep (their 1/(1-p) goes into the scales);
-//   dropout_dx_kernel     dX += s/(1-p) * (V A) * keep, the adapter's share of dX,
-//                         after the fused kernel wrote dY dequant(W) alone.
+//   dX += s/(1-p) * (V A) * keep, the adapter's share of dX, after the fused
+//                         kernel wrote dY dequant(W) alone: the masked-add epilogue
+//                         of the tensor-core GEMM V A (gemm_tc.cuh, kOutDropoutAdd),
+//                         which reads the keep bits the backward's mask kernel wrote.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -41,81 +43,45 @@ __device__ __forceinline__ uint4 dropout_words(uint64_t q, uint64_t seed, uint64
                        make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)));
 }
 
-// out = X with every dropped element replaced by +0 (bf16 bit patterns); four
-// elements (8 bytes, one Philox block) per thread and step.  n4 = M*K/4.
+// out = X with every dropped element replaced by +0 (bf16 bit patterns).  A
+// thread takes 16 consecutive elements (32 bytes, four Philox blocks) per
+// step, so four independent Philox chains are in flight per thread.
+// n16 = M*K/16 (M*K is a multiple of 64).  If `bits` is not NULL, bit j of
+// bits[q] is the keep decision of element 16 q + j (M*K/8 bytes), for
+// consumers that apply the same mask later without regenerating it.
 __global__ void __launch_bounds__(256)
-dropout_mask_kernel(const uint16_t* __restrict__ X, int64_t n4, uint32_t t, uint64_t seed, uint64_t offset,
-                    uint16_t* __restrict__ out) {
+dropout_mask_kernel(const uint16_t* __restrict__ X, int64_t n16, uint32_t t, uint64_t seed, uint64_t offset,
+                    uint16_t* __restrict__ out, uint16_t* __restrict__ bits) {
   griddep_wait();
-  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < n4;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < n16;
        q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 w = dropout_words(static_cast<uint64_t>(q), seed, offset);
-    uint2 x = __ldg(reinterpret_cast<const uint2*>(X) + q);
-    // element 4q is the low half of the first word
-    if (w.x < t) x.x &= 0xFFFF0000u;
-    if (w.y < t) x.x &= 0x0000FFFFu;
-    if (w.z < t) x.y &= 0xFFFF0000u;
-    if (w.w < t) x.y &= 0x0000FFFFu;
-    reinterpret_cast<uint2*>(out)[q] = x;
-  }
-  griddep_launch_dependents();
-}
-
-constexpr int kDxRows = 8;      // rows of dX per thread
-constexpr int kDxThreads = 256; // a thread owns 4 consecutive columns: 1024 columns per CTA
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// dX[m, k] = bf16(fp32(dX[m, k]) + scale * sum_j V[m, j] A[j, k]) where element
-// (m, k) is kept; dX unchanged where it was dropped.  V: bf16 M x r, A: bf16
-// r x K.  Shared memory: the CTA's kDxRows rows of V as fp32.
-__global__ void __launch_bounds__(kDxThreads)
-dropout_dx_kernel(uint16_t* __restrict__ dX, const uint16_t* __restrict__ V, const uint16_t* __restrict__ A,
-                  int64_t M, int64_t K, int r, float scale, uint32_t t, uint64_t seed, uint64_t offset) {
-  extern __shared__ float s_v[];
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kDxRows;
-  const int64_t k0 = (static_cast<int64_t>(blockIdx.x) * kDxThreads + threadIdx.x) * 4;
-  griddep_wait();
-  for (int i = threadIdx.x; i < kDxRows * r; i += kDxThreads) {
-    const int rr = i / r, j = i - rr * r;
-    s_v[i] = (m0 + rr < M) ? __uint_as_float(static_cast<uint32_t>(__ldg(V + (m0 + rr) * r + j)) << 16) : 0.f;
-  }
-  __syncthreads();
-  griddep_launch_dependents();
-  if (k0 >= K) return;
-  float acc[kDxRows][4];
+    uint4 w[4];
 #pragma unroll
-  for (int rr = 0; rr < kDxRows; ++rr) acc[rr][0] = acc[rr][1] = acc[rr][2] = acc[rr][3] = 0.f;
-  for (int j = 0; j < r; ++j) {
-    const uint2 a = __ldg(reinterpret_cast<const uint2*>(A + static_cast<int64_t>(j) * K + k0));
-    const float a0 = bf16_lo(a.x), a1 = bf16_hi(a.x), a2 = bf16_lo(a.y), a3 = bf16_hi(a.y);
+    for (int b = 0; b < 4; ++b) w[b] = dropout_words(static_cast<uint64_t>(4 * q + b), seed, offset);
+    const uint4* src = reinterpret_cast<const uint4*>(X) + 2 * q;
+    uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
+    uint32_t v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-    for (int rr = 0; rr < kDxRows; ++rr) {
-      const float v = s_v[rr * r + j];
-      acc[rr][0] = fmaf(v, a0, acc[rr][0]);
-      acc[rr][1] = fmaf(v, a1, acc[rr][1]);
-      acc[rr][2] = fmaf(v, a2, acc[rr][2]);
-      acc[rr][3] = fmaf(v, a3, acc[rr][3]);
+    for (int b = 0; b < 4; ++b) {
+      // Philox block b decides elements 4b .. 4b+3 (words 2b and 2b+1, low half first)
+      if (w[b].x < t) v[2 * b] &= 0xFFFF0000u;
+      if (w[b].y < t) v[2 * b] &= 0x0000FFFFu;
+      if (w[b].z < t) v[2 * b + 1] &= 0xFFFF0000u;
+      if (w[b].w < t) v[2 * b + 1] &= 0x0000FFFFu;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out) + 2 * q;
+    dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
+    if (bits) {
+      uint32_t k = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        k |= ((w[b].x >= t ? 1u : 0u) | (w[b].y >= t ? 2u : 0u) | (w[b].z >= t ? 4u : 0u) |
+              (w[b].w >= t ? 8u : 0u)) << (4 * b);
+      bits[q] = static_cast<uint16_t>(k);
     }
   }
-#pragma unroll
-  for (int rr = 0; rr < kDxRows; ++rr) {
-    const int64_t m = m0 + rr;
-    if (m >= M) break;
-    const int64_t e = m * K + k0;   // a multiple of 4: one Philox block
-    const uint4 w = dropout_words(static_cast<uint64_t>(e >> 2), seed, offset);
-    uint2* p = reinterpret_cast<uint2*>(dX + e);
-    uint2 d = *p;
-    const float o0 = w.x >= t ? bf16_lo(d.x) + scale * acc[rr][0] : bf16_lo(d.x);
-    const float o1 = w.y >= t ? bf16_hi(d.x) + scale * acc[rr][1] : bf16_hi(d.x);
-    const float o2 = w.z >= t ? bf16_lo(d.y) + scale * acc[rr][2] : bf16_lo(d.y);
-    const float o3 = w.w >= t ? bf16_hi(d.y) + scale * acc[rr][3] : bf16_hi(d.y);
-    __nv_bfloat162 h0 = __floats2bfloat162_rn(o0, o1), h1 = __floats2bfloat162_rn(o2, o3);
-    d.x = *reinterpret_cast<uint32_t*>(&h0);
-    d.y = *reinterpret_cast<uint32_t*>(&h1);
-    *p = d;
-  }
+  griddep_launch_dependents();
 }
 
 }  // namespace qlora

@@ -40,7 +40,11 @@ enum BSource : int {
   kBDeqK = 2,    // B = dequant(W) rows (weight row n = B row), K-major   (forward)
   kBDeqMN = 3,   // B = dequant(W)^T (weight row = reduction index), MN-major (dX)
 };
-enum OutMode : int { kOutBf16 = 0, kOutF32Partial = 1 };
+// kOutDropoutAdd: bf16 out(m, n) = bf16(fp32(out(m, n)) + drop_scale * D(m, n)) where bit
+// e = m * ld_out + n of the LoRA-dropout keep mask drop_bits (bit e & 31 of word e >> 5) is
+// set, out unchanged where it is clear (the adapter's share of dX under dropout).  In this mode the tensor map
+// tmA2 covers the output (bf16, box 64 x 128): the output tile comes in by TMA.
+enum OutMode : int { kOutBf16 = 0, kOutF32Partial = 1, kOutDropoutAdd = 2 };
 
 constexpr int kBK = 64;                 // reduction elements per stage (128 B of bf16)
 constexpr int kBM = 128;                // MMA M
@@ -62,21 +66,29 @@ struct GemmArgs {
   void* out;
   int64_t ld_out;         // elements between consecutive D rows
   int64_t split_stride;   // elements between splits (partial mode)
+  // kOutDropoutAdd: scale and keep bits
+  float drop_scale;
+  const uint32_t* drop_bits;
 };
 
-template <int BN, int NSTAGE, int BSRC, int NDW, int MH>
+template <int BN, int NSTAGE, int BSRC, int NDW, int MH, int OUT = kOutBf16>
 struct GemmSmem {
   static constexpr bool kDeq = (BSRC == kBDeqK || BSRC == kBDeqMN);
+  // kOutDropoutAdd: the output tile (bf16, MH x 128 rows x BN, 64-column boxes of 128-byte
+  // swizzled rows) is loaded by TMA while the MMAs run, and read back by the epilogue
+  static constexpr int kOutTileBytes = OUT == kOutDropoutAdd ? MH * kBM * BN * 2 : 0;
   static constexpr int kATileBytes = MH * kAHalfBytes;
   static constexpr int kBTileBytes = BN * kBK * 2;
   static constexpr int kPTileBytes = kDeq ? BN * kBK / 2 : 0;
   static constexpr int kAOff = 0;
   static constexpr int kBOff = kAOff + NSTAGE * kATileBytes;
-  static_assert(kBOff + NSTAGE * (kBTileBytes + kPTileBytes) + 1024 + 8 * (3 * NSTAGE + 1) + 16 <= 232448,
+  static_assert(kBOff + NSTAGE * (kBTileBytes + kPTileBytes) + kOutTileBytes + 1024 + 8 * (3 * NSTAGE + 2) + 16 <=
+                    232448,
                 "shared memory");
   static constexpr int kPOff = kBOff + NSTAGE * kBTileBytes;
-  static constexpr int kBarOff = kPOff + NSTAGE * kPTileBytes;
-  static constexpr int kNumBars = 3 * NSTAGE + 1;
+  static constexpr int kOutOff = kPOff + NSTAGE * kPTileBytes;   // 1024-byte aligned
+  static constexpr int kBarOff = kOutOff + kOutTileBytes;
+  static constexpr int kNumBars = 3 * NSTAGE + 2;   // full_tma, full_w, empty per stage; accum_full; out_full
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kDynBytes = kBytes + 1024;  // slack to align the base to 1024 B
@@ -155,7 +167,7 @@ __global__ void __launch_bounds__(64 + 32 * NDW, 1)
 qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                   const GemmArgs args) {
-  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH>;
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH, OUT>;
   constexpr bool kDeq = L::kDeq;
   constexpr int kATileBytes = L::kATileBytes;
   static_assert(MH == 1 || MH == 2, "MH");
@@ -173,6 +185,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint64_t* full_w = full_tma + NSTAGE;
   uint64_t* empty = full_w + NSTAGE;
   uint64_t* accum_full = empty + NSTAGE;
+  uint64_t* out_full = accum_full + 1;   // kOutDropoutAdd: the output tile landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -197,6 +210,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum_full, 1);
+    mbar_init(out_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -213,6 +227,16 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       if (n_lora > 0) { tma_prefetch_desc(&tmA2); tma_prefetch_desc(&tmB2); }
+      if (OUT == kOutDropoutAdd) {
+        // the output tile the epilogue updates (tmA2 maps the output: bf16, box 64 x 128)
+        mbar_arrive_expect_tx(out_full, static_cast<uint32_t>(L::kOutTileBytes));
+#pragma unroll
+        for (int h = 0; h < MH; ++h)
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_2d(smem + L::kOutOff + (h * (BN / 64) + c) * (kBM * 128), &tmA2, out_full, c0 + 64 * c,
+                        m0 + h * kBM);
+      }
       for (int t = 0; t < total; ++t) {
         const int s = t % NSTAGE;
         if (t >= NSTAGE && !mbar_wait(&empty[s], ((t / NSTAGE) - 1) & 1, abort_flag)) break;
@@ -397,6 +421,66 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
               if (total == 0) val = make_float4(0.f, 0.f, 0.f, 0.f);
               dst[(ch * 8 + i + row) & (BN / 4 - 1)] = val;
+            }
+          }
+        }
+      }
+    } else if (OUT == kOutDropoutAdd) {
+      // masked update of the output tile (MH == 1): this thread owns row q*32 + lane and
+      // the 32-column chunks ch = grp, grp + NDW/4, ...  Every keep word is loaded up
+      // front and two chunks leave TMEM per wait, so the latencies overlap.
+      static_assert(MH == 1, "masked update: one 128-row half");
+      constexpr int kChunks = BN / 32 / (NDW / 4);
+      static_assert(kChunks % 2 == 0, "chunks go in pairs");
+      const int q = warp & 3;
+      const int grp = (warp - 2) >> 2;
+      const int rl = q * 32 + lane;
+      const int row = m0 + rl;
+      const bool live = ok && total > 0 && row < args.m_rows;
+      uint32_t keep[kChunks];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        const int col = c0 + (grp + c * (NDW / 4)) * 32;
+        keep[c] = (live && col < args.n_cols)
+                      ? __ldg(args.drop_bits + ((static_cast<int64_t>(row) * args.ld_out + col) >> 5)) : 0u;
+      }
+      if (ok && total > 0) ok = mbar_wait(out_full, 0, abort_flag);
+      if (ok && total > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kChunks; c += 2) {
+          uint32_t v[2][32];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + (grp + (c + u) * (NDW / 4)) * 32,
+                               v[u]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int ch = grp + (c + u) * (NDW / 4);
+            const int col = c0 + ch * 32;
+            if (!live || col >= args.n_cols) continue;
+            const int64_t e = static_cast<int64_t>(row) * args.ld_out + col;   // a multiple of 32
+            // the current values, from the tile TMA brought in: row rl of 64-column box
+            // ch / 2, 16-byte chunks (ch % 2) * 4 + i at (chunk ^ (rl & 7)) * 16
+            const uint32_t box = smem_u32(smem + L::kOutOff + (ch / 2) * (kBM * 128)) + rl * 128;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + e);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t c16 = static_cast<uint32_t>((ch & 1) * 4 + i);
+              const uint4 d = ld_shared_v4(box + ((c16 ^ static_cast<uint32_t>(rl & 7)) << 4));
+              const uint32_t in[4] = {d.x, d.y, d.z, d.w};
+              uint32_t o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int b = 8 * i + 2 * j;   // element e + b (low half), e + b + 1 (high half)
+                const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
+                const float x0 = ((keep[c + u] >> b) & 1u) ? lo + args.drop_scale * __uint_as_float(v[u][b]) : lo;
+                const float x1 = ((keep[c + u] >> (b + 1)) & 1u) ? hi + args.drop_scale * __uint_as_float(v[u][b + 1]) : hi;
+                __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+                o[j] = *reinterpret_cast<uint32_t*>(&hb);
+              }
+              dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
         }

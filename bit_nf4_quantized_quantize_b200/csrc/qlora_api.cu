@@ -241,7 +241,7 @@ int launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaSt
 template <int BN, int NSTAGE, bool A_MN, int BSRC, int OUT, int NDW, int MH = 1>
 int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                 const CUtensorMap& b2, const GemmArgs& args, cudaStream_t st, int dev) {
-  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH>;
+  using L = GemmSmem<BN, NSTAGE, BSRC, NDW, MH, OUT>;
   auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW, MH>;
   // the adapter slices must fit in the first pass over the stages
   if (args.n_lora > NSTAGE) return QLORA_ERR_UNSUPPORTED_SHAPE;
@@ -253,7 +253,8 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
     }
     attr_set[dev] = true;
   }
-  const int kind = (BSRC == kBDeqK) ? QLORA_KERNEL_FWD
+  const int kind = (OUT == kOutDropoutAdd) ? QLORA_KERNEL_DROPOUT
+                 : (BSRC == kBDeqK) ? QLORA_KERNEL_FWD
                  : (BSRC == kBDeqMN) ? QLORA_KERNEL_DX
                  : A_MN ? QLORA_KERNEL_GRAD_GEMM : QLORA_KERNEL_LORA_GEMM;
   return timed(kind, st, [&] {
@@ -376,12 +377,13 @@ int run_decode(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t us, v, vs, u, xm, total;
+  size_t us, v, vs, u, xm, bits, total;
 };
 
 // bf16 scratch of M x r each: s*U (forward adapter operand), V and s*V
 // (backward), U (recomputed when the caller passes no saved U).
-// With dropout, xm holds the masked adapter input X * keep (bf16 M x K).
+// With dropout, xm holds the masked adapter input X * keep (bf16 M x K) and
+// bits the keep mask, one bit per element (M x K / 8 bytes).
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms, bool dropout = false) {
   (void)N; (void)num_sms;
   WsLayout w;
@@ -391,7 +393,8 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int num_sms, bool dro
   w.vs = w.v + mr;
   w.u = w.vs + mr;
   w.xm = w.u + mr;
-  w.total = w.xm + (dropout ? a256(static_cast<size_t>(M) * K * 2) : 0);
+  w.bits = w.xm + (dropout ? a256(static_cast<size_t>(M) * K * 2) : 0);
+  w.total = w.bits + (dropout ? a256(static_cast<size_t>(M) * K / 8) : 0);
   return w;
 }
 
@@ -607,13 +610,15 @@ bool make_dropout(float p, uint64_t seed, uint64_t offset, DropoutSpec* d) {
 }
 
 // X * keep (bf16 M x K) into `out`.
+// out = X * keep; bits (or NULL) receives the keep mask, one bit per element.
 int launch_dropout_mask(const uint16_t* X, int64_t M, int64_t K, const DropoutSpec& d, uint16_t* out, int sms,
-                        cudaStream_t st) {
-  const int64_t n4 = M * K / 4;
-  const int64_t want = (n4 + 255) / 256;
+                        cudaStream_t st, uint16_t* bits = nullptr) {
+  const int64_t n16 = M * K / 16;   // K % 64 == 0
+  const int64_t want = (n16 + 255) / 256;
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   return timed(QLORA_KERNEL_DROPOUT, st, [&] {
-    return launch_ex(dropout_mask_kernel, dim3(blocks), dim3(256), 0, st, 1, 1, X, n4, d.t, d.seed, d.offset, out);
+    return launch_ex(dropout_mask_kernel, dim3(blocks), dim3(256), 0, st, 1, 1, X, n16, d.t, d.seed, d.offset, out,
+                     bits);
   });
 }
 
@@ -1029,7 +1034,8 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   const uint16_t* Xa = X;
   if (dr.on) {
     uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
-    if (int rc = launch_dropout_mask(X, M, K, dr, Xm, sms, st)) return rc;
+    uint16_t* keep_bits = reinterpret_cast<uint16_t*>(ws + L.bits);   // read by the masked dX term
+    if (int rc = launch_dropout_mask(X, M, K, dr, Xm, sms, st, keep_bits)) return rc;
     Xa = Xm;
   }
   // U (from the forward, or recomputed)
@@ -1056,8 +1062,8 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     }
   }
   // dX = dY dequant(W) + (s V) A; with dropout the adapter term is masked, so
-  // the fused kernel computes dY dequant(W) alone and dropout_dx_kernel adds
-  // s/(1-p) (V A) where the input was kept
+  // the fused kernel computes dY dequant(W) alone and a tensor-core GEMM V A
+  // adds s/(1-p) (V A) where the input was kept (masked-add epilogue)
   if (dX) {
     GemmArgs g{};
     g.m_rows = static_cast<int>(M);
@@ -1098,14 +1104,25 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     }
     if (rc) return rc;
     if (dr.on) {
-      const dim3 grid(static_cast<unsigned>((K + 4 * kDxThreads - 1) / (4 * kDxThreads)),
-                      static_cast<unsigned>((M + kDxRows - 1) / kDxRows));
-      const size_t smem = sizeof(float) * kDxRows * static_cast<size_t>(r);
-      const float scale = s * dr.inv;
-      rc = timed(QLORA_KERNEL_DROPOUT, st, [&] {
-        return launch_ex(dropout_dx_kernel, grid, dim3(kDxThreads), smem, st, 1, 1, dX, V, A, M,
-                         static_cast<int64_t>(K), r, scale, dr.t, dr.seed, dr.offset);
-      });
+      // D = V A: A operand V (M x r, K-major), B operand the adapter's A (r x K, MN-major);
+      // r is one to four reduction steps of 64 (zero-filled past r)
+      CUtensorMap tv, ta, tdx;
+      if (!map_bf16(&tv, V, M, r, 64, 128) || !map_bf16(&ta, A, r, K, 64, 64) || !map_bf16(&tdx, dX, M, K, 64, 128))
+        return QLORA_ERR_CUDA;
+      GemmArgs gd{};
+      gd.m_rows = static_cast<int>(M);
+      gd.n_cols = K;
+      gd.k_steps = rpad / 64;
+      gd.steps_per_split = gd.k_steps;
+      gd.n_lora = 0;
+      gd.out = dX;
+      gd.ld_out = K;
+      gd.drop_scale = s * dr.inv;
+      gd.drop_bits = reinterpret_cast<const uint32_t*>(ws + L.bits);
+      // 128 x 128 tiles, one stage, four epilogue warps: two CTAs per SM, so one CTA's
+      // loads overlap another's masked update
+      const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 127) / 128), 1);
+      rc = launch_gemm<128, 1, false, kBTmaMN, kOutDropoutAdd, 4, 1>(grid, tv, ta, tdx, ta, gd, st, dev);
       if (rc) return rc;
     }
   }
