@@ -78,6 +78,18 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def sync_adapter_grads(dA, dB, world: int) -> None:
+    """The data-parallel exchange of a step: every rank holds the gradients of its own token
+    shard, and the adapter's gradients are their sum over ranks (the frozen NF4 weight and the
+    adapter are replicated; dX stays with its shard).  One all-reduce each of dA and dB
+    (r (N + K) fp32), on the stream the kernels ran on."""
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    dist.all_reduce(dA, op=dist.ReduceOp.SUM)
+    dist.all_reduce(dB, op=dist.ReduceOp.SUM)
+
+
 def job_throughput(world: int, units_per_rank: float, ms: float, scale: float = 1e12) -> float:
     """Whole-job rate: the units all ranks processed (replicas: world x per rank) / the step time."""
     return world * units_per_rank / (ms * 1e-3) / scale
@@ -648,6 +660,7 @@ def run_ours(args, rank, world, local_rank):
         q.qlora_linear_fwd(codes, q8, s2, N, K, Xd, Ad, Bd, alpha, Y=Y, U_save=U, workspace=ws)
         q.qlora_linear_bwd(codes, q8, s2, N, K, Xd, Ad, Bd, alpha, dYd, U_saved=U, dX=dX, dA=dA, dB=dB,
                            workspace=ws)
+        sync_adapter_grads(dA, dB, world)   # N > 1: sum the adapter gradients over the token shards
 
     def barrier():
         if world > 1:
@@ -791,7 +804,9 @@ def run_ours(args, rank, world, local_rank):
                    "N": N, "K": K, "M": M, "r": r, "alpha": alpha,
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a {L2_FLUSH_BYTES >> 20} MiB read "
                          "that writes back the dirty lines; outside the step events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+                   "parallelism": (f"data parallel x{world}: token shards, replicated NF4 weight and adapter, "
+                                   "dA and dB summed over ranks (NCCL all-reduce) every step")
+                                  if world > 1 else "1 GPU"},
         "roofline": roof,
         "quantize": {"gbs": qburst["gbs"], "peak_gbs": peaks["hbm_gbs"], "frac": qburst["frac"],
                      "ms_per_launch": qburst["ms_per_launch"], "timing": qburst["how"],
