@@ -50,6 +50,18 @@
  *   no element (n_out == 0 or k_in == 0) makes the quantizers, the
  *   dequantizer and the merge no-ops whose pointers may be NULL.  The layer
  *   itself needs N, K >= 64.
+ * - Launch order.  Every kernel is launched with programmatic stream
+ *   serialisation, and the first kernel of a call waits for the previous work
+ *   on the stream to complete before it reads anything.  Stream order holds as
+ *   usual: a call reads its inputs after all earlier work on the stream and
+ *   its outputs are complete for all later work.  One exception is a later
+ *   kernel that the caller launches with programmatic stream serialisation of
+ *   its own.  It may start before the call's last kernel ends, and it must
+ *   wait for its grid dependency (cudaGridDependencySynchronize) before it
+ *   touches the call's outputs.  Inside a call, kernels overlap where their
+ *   data allow: the fused kernels start on the adapter products' free SMs, and
+ *   the backward's gradient kernel runs on a second, library-owned stream of
+ *   the device, joined back before the call's last kernel completes.
  * - Return value: QLORA_OK (0) or a negative QLORA_ERR_* code.  Errors raised
  *   on the device after a call returned (a bounded wait inside a kernel that
  *   gave up) are latched in a device flag and reported by qlora_device_status.
