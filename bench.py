@@ -12,9 +12,11 @@ Metric: algorithmic fwd+bwd FLOP of the step / device time of the step
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 runs under torchrun as independent replicas (one process per GPU, no
-collective on the data path; weak scaling).  --impl reference times the CPU
-oracle on the same workload (a bounded sample of it per step).
+N > 1 runs under torchrun, data parallel: one process per GPU, each with its
+own tokens of the same shape (weak scaling) and a replica of the weight and
+the adapter; the step ends with an NCCL all-reduce of dA and dB.  --impl
+reference times the CPU oracle on the same workload (a bounded sample of it
+per step).
 """
 from __future__ import annotations
 
@@ -749,24 +751,52 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
     d2h = sum(t.numel() * t.element_size() for t in (hY, hdX, hdA, hdB))
     e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+    # Uploads and downloads run on their own streams so that the two copy
+    # directions overlap each other and the kernels: W goes up first (the
+    # quantizer needs only W), then X, A, B (the forward), then dY (the
+    # backward); Y comes down while dY goes up and the backward runs, then
+    # dX, dA, dB.  The library calls stay on the current stream.
+    cur = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     barrier()
     torch.cuda.synchronize()
     for i in range(n_e2e):
         flush(float(i))
-        e_ev[i][0].record()
-        W.copy_(hW, non_blocking=True)
-        X.copy_(hX, non_blocking=True)
-        A.copy_(hA, non_blocking=True)
-        B.copy_(hB, non_blocking=True)
-        dY.copy_(hdY, non_blocking=True)
-        step()
-        hY.copy_(Y, non_blocking=True)
-        hdX.copy_(dX, non_blocking=True)
-        hdA.copy_(dA, non_blocking=True)
-        hdB.copy_(dB, non_blocking=True)
-        e_ev[i][1].record()
+        e_ev[i][0].record(cur)
+        up.wait_stream(cur)
+        with torch.cuda.stream(up):
+            W.copy_(hW, non_blocking=True)
+            w_up = up.record_event()
+            X.copy_(hX, non_blocking=True)
+            A.copy_(hA, non_blocking=True)
+            B.copy_(hB, non_blocking=True)
+            x_up = up.record_event()
+            dY.copy_(hdY, non_blocking=True)
+            dy_up = up.record_event()
+        cur.wait_event(w_up)
+        q.qlora_quantize_nf4_dq(W, codes, q8, s2)
+        cur.wait_event(x_up)
+        q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, Y=Y, U_save=U, workspace=ws)
+        down.wait_stream(cur)
+        with torch.cuda.stream(down):
+            hY.copy_(Y, non_blocking=True)
+        cur.wait_event(dy_up)
+        q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U, dX=dX, dA=dA, dB=dB,
+                           workspace=ws)
+        sync_adapter_grads(dA, dB, world)
+        down.wait_stream(cur)
+        with torch.cuda.stream(down):
+            hdX.copy_(dX, non_blocking=True)
+            hdA.copy_(dA, non_blocking=True)
+            hdB.copy_(dB, non_blocking=True)
+        cur.wait_stream(down)
+        e_ev[i][1].record(cur)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / n_e2e, world, dev)
+    # the copies must have carried the step's own results
+    if not (torch.equal(hY, Y.cpu()) and torch.equal(hdX, dX.cpu()) and torch.equal(hdA, dA.cpu())
+            and torch.equal(hdB, dB.cpu())):
+        raise RuntimeError("end-to-end results differ from the device-resident step's")
 
     if rank != 0:
         return
@@ -817,7 +847,10 @@ def run_ours(args, rank, world, local_rank):
         "kernels": per_step,
         "gpu_launches": launches,
         "e2e": {"value": job_throughput(world, fl, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "copies": "pinned host buffers; uploads and downloads on two copy streams, overlapped with "
+                          "each other and the kernels (W, then X/A/B, then dY up; Y down after the forward, "
+                          "dX/dA/dB after the backward)"},
         "clocks": clocks,
     }
     line["decode"] = run_decode(q, dev, peaks)
