@@ -5,8 +5,8 @@ identical to the GPU's), dequantizes to bf16 and evaluates the layer in fp64 on
 the exact bf16 operands.  Tolerance: relative L2 <= 4e-3 on every output and
 gradient.  Cases span several tiles with ragged tails in M, N and K, adapter
 ranks from 8 to 256 (one to four adapter slices), the tiny and decode
-workloads in full, and the 4096^3 training workload, the 7B down projection and
-the 65B 22016 x 8192 linear on sampled rows (dA, dB in full).
+workloads in full, and on sampled rows (dA, dB in full) the 4096^3 training
+workload, the three weight shapes of the 7B stack and both 65B linears.
 """
 import numpy as np
 import pytest
@@ -92,6 +92,24 @@ def test_llama7b_down_proj_sampled_rows():
     """The 7B stack's down projection (4096 x 11008, outlier weights), M = 2048."""
     inp = synth.layer_inputs("llama7b", layer=6)
     rows = np.arange(0, 2048, 97)
+    run_case(inp, rows=rows)
+
+
+@pytest.mark.parametrize("layer", [0, 4])
+def test_llama7b_attention_and_gate_sampled_rows(layer):
+    """The 7B stack's 4096 x 4096 projection and its 11008 x 4096 gate projection (N not a
+    multiple of the 512-wide pair tile), outlier weights, M = 2048, at full size in the bench's
+    launch configuration: Y, U and dX on sampled rows, dA and dB in full."""
+    inp = synth.layer_inputs("llama7b", layer=layer)
+    rows = np.unique(np.concatenate([np.arange(0, 2048, 89), [2047]]))
+    run_case(inp, rows=rows)
+
+
+def test_llama65b_square_sampled_rows():
+    """The 65B config's 8192 x 8192 linear (Student-t weights), M = 8192, r = 64, at full size:
+    Y, U and dX on sampled rows, dA and dB in full."""
+    inp = synth.layer_inputs("llama65b", layer=0)
+    rows = np.unique(np.concatenate([np.arange(0, 8192, 331), [8191]]))
     run_case(inp, rows=rows)
 
 
