@@ -113,6 +113,9 @@ def _ptr(t):
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {stream.device}; the library launches on the current device "
+                         f"cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -128,6 +131,9 @@ def _dev(t, dtype, name, shape=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}; the library launches on the current device "
+                         f"cuda:{torch.cuda.current_device()} (use torch.cuda.device)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -252,7 +258,7 @@ def qlora_workspace_bytes(M: int, n_out: int, k_in: int, r: int) -> int:
 
 
 def _nbytes(ws):
-    return 0 if ws is None else ws.numel()
+    return 0 if ws is None else ws.numel() * ws.element_size()
 
 
 def _workspace(ws, M, N, K, r, device):
@@ -263,6 +269,8 @@ def _workspace(ws, M, N, K, r, device):
         raise QloraError(-2, "qlora_workspace_bytes")
     if ws is None:
         ws = torch.empty(need, dtype=torch.uint8, device=device)
+    else:
+        _dev(ws, ws.dtype, "workspace")
     return ws
 
 
@@ -343,6 +351,8 @@ def _workspace_dropout(ws, M, N, K, r, device):
         raise QloraError(-2, "qlora_workspace_bytes_dropout")
     if ws is None:
         ws = torch.empty(need, dtype=torch.uint8, device=device)
+    else:
+        _dev(ws, ws.dtype, "workspace")
     return ws
 
 

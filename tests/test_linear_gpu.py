@@ -226,3 +226,23 @@ def test_empty_batch_and_empty_weight():
         assert c.numel() == 0 and qq.numel() == 0 and ss.numel() == 0
         assert q.qlora_dequant(c, qq, ss, *shape).numel() == 0
     assert q.qlora_device_status() == 0
+
+
+def test_caller_workspace_of_any_dtype_and_too_small():
+    """A caller workspace is counted in bytes whatever its dtype: a float32 buffer of the
+    required size works and gives the same bits as the binding's own; one byte short is
+    refused with the workspace error before any launch."""
+    inp = synth.layer_inputs("tiny", M=300, shape=(512, 768), r=16, seed=41)
+    N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    X, A, B = (to_dev_bf16(inp[k]) for k in ("X", "A", "B"))
+    need = q.qlora_workspace_bytes(M, N, K, r)
+    ws32 = torch.empty((need + 3) // 4, dtype=torch.float32, device="cuda")
+    Y0 = q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha)
+    Y1 = q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, workspace=ws32)
+    assert torch.equal(Y0, Y1)
+    short = torch.empty(need - 1, dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QloraError) as e:
+        q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, workspace=short)
+    assert e.value.code == -5
+    assert q.qlora_device_status() == 0
