@@ -235,12 +235,12 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 
 def dropout_threshold(p: float) -> int:
-    """Integer keep threshold floor(p * 2^32) of the fp32 value of p (clamped to 2^32 - 1);
-    an element is kept iff its word >= it."""
+    """Integer keep threshold floor(p * 2^16) of the fp32 value of p (at most 2^16 - 1 for
+    p < 1); an element is kept iff its 16-bit half word >= it."""
     p32 = float(np.float32(p))
     if not 0.0 <= p32 < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(int(np.floor(p32 * 4294967296.0)), 0xFFFFFFFF)
+    return int(np.floor(p32 * 65536.0))
 
 
 def dropout_keep(M: int, K: int, p: float, seed: int, offset: int) -> np.ndarray:

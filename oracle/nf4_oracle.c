@@ -385,20 +385,23 @@ void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t
     out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
 }
 
-/* Keep decision of element e (row-major index m*K + k of X): word (e & 3)  */
-/* of Philox4x32-10 with counter (lo32(e>>2), hi32(e>>2), lo32(offset),     */
-/* hi32(offset)) and key (lo32(seed), hi32(seed)); the element is kept when */
-/* that word is >= t, t = floor(p * 2^32) (the caller's integer threshold). */
+/* Keep decision of element e (row-major index m*K + k of X).  One block of */
+/* Philox4x32-10, counter (lo32(e>>3), hi32(e>>3), lo32(offset),            */
+/* hi32(offset)) and key (lo32(seed), hi32(seed)), decides 8 elements: e    */
+/* reads the 16-bit half (e & 1) (0 = the low half) of word ((e >> 1) & 3) */
+/* and is kept when that half is >= t, t = floor(p * 2^16) (the caller's    */
+/* integer threshold), so the drop probability is t / 2^16.                 */
 void oracle_dropout_keep(int64_t M, int64_t K, uint32_t t, uint64_t seed, uint64_t offset, uint8_t* keep) {
     const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
 #pragma omp parallel for schedule(static)
-    for (int64_t q = 0; q < (M * K + 3) / 4; ++q) {
+    for (int64_t q = 0; q < (M * K + 7) / 8; ++q) {
         uint32_t ctr[4] = {(uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)offset, (uint32_t)(offset >> 32)};
         uint32_t w[4];
         oracle_philox4x32_10(ctr, key, w);
-        for (int j = 0; j < 4; ++j) {
-            int64_t e = q * 4 + j;
-            if (e < M * K) keep[e] = w[j] >= t ? 1 : 0;
+        for (int j = 0; j < 8; ++j) {
+            int64_t e = q * 8 + j;
+            uint32_t half = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+            if (e < M * K) keep[e] = half >= t ? 1 : 0;
         }
     }
 }

@@ -531,12 +531,17 @@ def test_dropout_keep_rate_and_layout():
         n = keep.size
         assert abs(keep.mean() - (1 - p)) <= 5 * np.sqrt(p * (1 - p) / n)
     assert np.all(oracle.dropout_keep(8, 64, 0.0, seed=1, offset=0) == 1)
-    # element e = m*K + k uses word e & 3 of the block at counter (e >> 2, offset)
+    # 16-bit thresholds: floor(p * 2^16) of the fp32 p; the largest fp32 below 1 gives 2^16 - 1
+    assert oracle.dropout_threshold(0.25) == 16384 and oracle.dropout_threshold(0.05) == 3276
+    assert oracle.dropout_threshold(float(np.nextafter(np.float32(1), np.float32(0)))) == 65535
+    # element e = m*K + k uses the 16-bit half e & 1 (low half first) of word (e >> 1) & 3 of
+    # the block at counter (e >> 3, offset)
     keep = oracle.dropout_keep(4, 64, 0.25, seed=0x1122334455667788, offset=0x99)
     t = oracle.dropout_threshold(0.25)
-    for e in (0, 1, 2, 3, 4, 77, 255):
-        w = oracle.philox4x32_10([e >> 2, 0, 0x99, 0], [0x55667788, 0x11223344])
-        assert keep.reshape(-1)[e] == (1 if w[e & 3] >= t else 0)
+    for e in (0, 1, 2, 3, 4, 5, 6, 7, 8, 77, 255):
+        w = oracle.philox4x32_10([e >> 3, 0, 0x99, 0], [0x55667788, 0x11223344])
+        half = (int(w[(e >> 1) & 3]) >> (16 * (e & 1))) & 0xFFFF
+        assert keep.reshape(-1)[e] == (1 if half >= t else 0)
     # another offset gives another mask
     assert not np.array_equal(oracle.dropout_keep(64, 64, 0.5, 3, 0), oracle.dropout_keep(64, 64, 0.5, 3, 1))
 
