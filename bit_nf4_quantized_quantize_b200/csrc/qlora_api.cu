@@ -585,8 +585,8 @@ int run_lora_down(const uint16_t* X, int64_t M, int64_t K, const uint16_t* Amat,
 }
 
 // ------------------------------------------------------------------ LoRA dropout
-// Dropout on the adapter input (dropout.cuh): integer keep threshold t =
-// floor(p * 2^32) and scale inv = fp32(1 / (1 - p)), both from the fp32 p.
+// Dropout on the adapter input (dropout.cuh): 16-bit keep threshold t =
+// floor(p * 2^16) and scale inv = fp32(1 / (1 - p)), both from the fp32 p.
 struct DropoutSpec {
   bool on = false;
   uint32_t t = 0;
@@ -600,9 +600,8 @@ bool make_dropout(float p, uint64_t seed, uint64_t offset, DropoutSpec* d) {
   *d = DropoutSpec{};
   if (p == 0.f) return true;
   const double pd = static_cast<double>(p);
-  const double tt = std::floor(pd * 4294967296.0);
   d->on = true;
-  d->t = tt >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(tt);
+  d->t = static_cast<uint32_t>(std::floor(pd * 65536.0));   // <= 0xFFFF for p < 1
   d->inv = static_cast<float>(1.0 / (1.0 - pd));
   d->seed = seed;
   d->offset = offset;
@@ -615,7 +614,23 @@ int launch_dropout_mask(const uint16_t* X, int64_t M, int64_t K, const DropoutSp
                         cudaStream_t st, uint16_t* bits = nullptr) {
   const int64_t n16 = M * K / 16;   // K % 64 == 0
   const int64_t want = (n16 + 255) / 256;
-  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  // one round of resident blocks: the grid-stride loop then ends evenly on every SM
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  static int resident[kMaxDevices];   // blocks of 256 threads per SM, 0 = not yet asked
+  if (resident[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dropout_mask_kernel, 256, 0) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    resident[dev] = n;
+  }
+  const unsigned blocks =
+      static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * resident[dev]));
   return timed(QLORA_KERNEL_DROPOUT, st, [&] {
     return launch_ex(dropout_mask_kernel, dim3(blocks), dim3(256), 0, st, 1, 1, X, n16, d.t, d.seed, d.offset, out,
                      bits);

@@ -263,10 +263,12 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
  *   Y  = X dequant(W)^T + s (Xd A^T) B^T,  U = Xd A^T,  Xd = X * keep / (1 - p)
  *   dX = dY dequant(W) + s ((dY B) A) * keep / (1 - p)
  *   dA = s (dY B)^T Xd,  dB = s dY^T U
- * keep(e) for element e = m*K + k of X: word (e & 3) of Philox4x32-10 (Salmon
- * et al., SC'11) at counter (lo32(e>>2), hi32(e>>2), lo32(offset),
- * hi32(offset)) with key (lo32(seed), hi32(seed)) is >= floor(p * 2^32); the
- * scale is fp32(1 / (1 - p)); both are taken from the fp32 p.  p must be in
+ * keep(e) for element e = m*K + k of X: the 16-bit half (e & 1), low half
+ * first, of word ((e >> 1) & 3) of Philox4x32-10 (Salmon et al., SC'11) at
+ * counter (lo32(e>>3), hi32(e>>3), lo32(offset), hi32(offset)) with key
+ * (lo32(seed), hi32(seed)) is >= floor(p * 2^16), so the drop probability is
+ * within 2^-16 of p; the scale is fp32(1 / (1 - p)); both are taken from the
+ * fp32 p.  p must be in
  * [0, 1) (else QLORA_ERR_INVALID_ARG); p == 0 is exactly the plain call.
  * Pass the same (p, seed, offset) to the forward and the backward of a step.
  * The workspace must hold qlora_workspace_bytes_dropout(M, N, K, r) bytes
