@@ -218,7 +218,7 @@ def oracle_step(inp, M_s):
     """One sampled step on the CPU oracle: quantize the whole W, then fwd + bwd on M_s tokens."""
     import oracle
     from bit_nf4_quantized_quantize_b200 import synth
-    N, K, r, alpha = inp["N"], inp["K"], inp["r"], inp["alpha"]
+    N, K, alpha = inp["N"], inp["K"], inp["alpha"]
     t0 = time.perf_counter()
     codes, q8, s2, _ = oracle.quantize_nf4_dq(inp["W"].reshape(-1))
     t1 = time.perf_counter()
@@ -824,7 +824,6 @@ def run_ours(args, rank, world, local_rank):
     qk = kern.get("quantize")
     quant_gbs = quant_bytes(N, K) / (qk[0] / qk[1] * 1e-3) / 1e9 if qk else None
     qburst = run_quantize_burst(q, dev, W, peaks)
-    fwd_ms = sum(per_step[k]["ms_per_step"] for k in per_step if k in ("lora_gemm", "lora_reduce", "fwd_fused")) / 1
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
