@@ -720,6 +720,26 @@ AuxStream* aux_stream(int dev) {
   return &a;
 }
 
+// Whether work of a call on stream st may go to the second stream: it must
+// not be inside a stream capture other than st's own.  A capture that st
+// runs takes the second stream in through the fork event (and the graph then
+// keeps the two branches); a capture that another caller left open on it
+// must not receive this call's kernel, which then stays on st.
+bool aux_usable(cudaStream_t st, cudaStream_t aux) {
+  cudaStreamCaptureStatus sa = cudaStreamCaptureStatusNone, ss = cudaStreamCaptureStatusNone;
+  unsigned long long ida = 0, ids = 0;
+  if (cudaStreamGetCaptureInfo(aux, &sa, &ida) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (sa == cudaStreamCaptureStatusNone) return true;
+  if (cudaStreamGetCaptureInfo(st, &ss, &ids) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return sa == cudaStreamCaptureStatusActive && ss == cudaStreamCaptureStatusActive && ids == ida;
+}
+
 // Persistent quantizer: one CTA per SM (its shared-memory ring fills most of
 // the SM), never more CTAs than groups.
 template <int kMode>
@@ -1065,12 +1085,14 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   }
   // The gradient kernel goes to the device's second stream, forked here and
   // launched after dX so that dX's CTAs are queued first; with per-kernel
-  // timing on, every kernel stays on the caller's stream (each timed alone).
+  // timing on, every kernel stays on the caller's stream (each timed alone),
+  // and so does it while another caller's capture holds the second stream.
   std::unique_lock<std::mutex> aux_lk(g_aux_mu, std::defer_lock);
   AuxStream* aux = nullptr;
   if (!g_timing_on && dX) {
     aux_lk.lock();
     aux = aux_stream(dev);
+    if (aux && !aux_usable(st, aux->s)) aux = nullptr;
     if (aux && cudaEventRecord(aux->fork, st) != cudaSuccess) {
       cudaGetLastError();
       return QLORA_ERR_CUDA;

@@ -247,6 +247,14 @@ int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const floa
  *   recompute U = X A^T here.  dX may be NULL (not computed).  dA and dB are
  *   overwritten (not accumulated).  The reductions over M are deterministic:
  *   the same inputs give bit-identical dA and dB on every call.
+ *
+ *   With dX requested, the kernel for dA and dB runs on a second stream that
+ *   the library keeps per device, forked from `stream` by an event and joined
+ *   back before the call returns, so the caller sees plain stream order.  A
+ *   stream capture on `stream` takes that branch into its graph.  While the
+ *   second stream belongs to a capture of another stream, calls outside that
+ *   capture keep the kernel on their own stream.  The call is safe from
+ *   several host threads.
  */
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      int64_t n_out, int64_t k_in,

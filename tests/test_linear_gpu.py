@@ -246,3 +246,55 @@ def test_caller_workspace_of_any_dtype_and_too_small():
         q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, workspace=short)
     assert e.value.code == -5
     assert q.qlora_device_status() == 0
+
+
+def test_backward_on_two_streams_and_inside_a_graph_capture():
+    """The backward forks its gradient kernel to a second stream of the library's.  Two
+    backward calls in flight on two streams, and a backward captured in a CUDA graph while an
+    uncaptured one runs on another stream, give the bits of a plain call.  The uncaptured
+    call must stay out of the capture that holds the second stream."""
+    inp = synth.layer_inputs("tiny", M=300, shape=(512, 768), r=16, seed=55)   # CTA-pair path
+    N, K, M, r, alpha = inp["N"], inp["K"], inp["M"], inp["r"], inp["alpha"]
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
+    U = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, alpha, U_save=U)
+    ref = q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U)
+    torch.cuda.synchronize()
+
+    def bufs():
+        out = (torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda"),
+               torch.full((r, K), float("nan"), device="cuda"), torch.full((N, r), float("nan"), device="cuda"))
+        return out + (torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda"),)
+
+    def bwd(b):
+        q.qlora_linear_bwd(codes, q8, s2, N, K, X, A, B, alpha, dY, U_saved=U, dX=b[0], dA=b[1], dB=b[2],
+                           workspace=b[3])
+
+    def same(b):
+        return all(torch.equal(x, y) for x, y in zip(b[:3], ref))
+
+    s_a, s_b = torch.cuda.Stream(), torch.cuda.Stream()
+    b1, b2 = bufs(), bufs()
+    torch.cuda.synchronize()
+    for s, b in ((s_a, b1), (s_b, b2)):
+        with torch.cuda.stream(s):
+            bwd(b)
+    torch.cuda.synchronize()
+    assert same(b1) and same(b2)
+
+    c1, c2 = bufs(), bufs()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s_a, capture_error_mode="relaxed"):
+        bwd(c1)                      # captured: the second stream joins this capture
+        with torch.cuda.stream(s_b):
+            bwd(c2)                  # runs now, outside the capture
+    torch.cuda.synchronize()
+    assert same(c2)
+    assert torch.isnan(c1[1]).all()  # the captured call has not run yet
+    g.replay()
+    torch.cuda.synchronize()
+    assert same(c1)
+    del g
+    assert q.qlora_device_status() == 0
