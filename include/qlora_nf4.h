@@ -253,8 +253,8 @@ int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* q8, const floa
  *   back before the call returns, so the caller sees plain stream order.  A
  *   stream capture on `stream` takes that branch into its graph.  While the
  *   second stream belongs to a capture of another stream, calls outside that
- *   capture keep the kernel on their own stream.  The call is safe from
- *   several host threads.
+ *   capture keep the kernel on their own stream.  Calls from several host
+ *   threads take turns on the second stream under a lock.
  */
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      int64_t n_out, int64_t k_in,
