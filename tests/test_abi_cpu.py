@@ -118,3 +118,27 @@ def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(ValueError):
         q.qlora_quantize_nf4_dq(torch.zeros(64, 64))
+
+
+def test_dropout_host_validation_without_gpu(lib):
+    """The dropout entry points refuse p outside [0, 1) (NaN included) and bad shapes before
+    touching any device; an empty batch is valid without buffers; the dropout workspace holds
+    the plain one plus the masked input and its keep bits."""
+    P = 1 << 20
+    null = None
+    for p in (-0.1, 1.0, 1.5, float("nan")):
+        assert lib.qlora_linear_fwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                            p, 1, 0, _p(P), null, _p(P), 1 << 30, null) == -1
+        assert lib.qlora_linear_bwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                            p, 1, 0, _p(P), null, null, _p(P), _p(P), _p(P), 1 << 30,
+                                            null) == -1
+        assert lib.qlora_dropout_apply(_p(P), 16, 256, p, 1, 0, _p(P), null) == -1
+    assert lib.qlora_dropout_apply(_p(P), 16, 100, 0.1, 1, 0, _p(P), null) == -2   # K % 64
+    assert lib.qlora_dropout_apply(_p(P), -1, 256, 0.1, 1, 0, _p(P), null) == -2
+    assert lib.qlora_dropout_apply(null, 0, 256, 0.1, 1, 0, null, null) == 0       # empty batch
+    assert lib.qlora_dropout_apply(null, 16, 256, 0.1, 1, 0, _p(P), null) == -1
+    assert lib.qlora_dropout_apply(_p(P + 2), 16, 256, 0.1, 1, 0, _p(P), null) == -2
+    M, N, K, r = 4096, 4096, 4096, 64
+    plain = q.qlora_workspace_bytes(M, N, K, r)
+    assert q.qlora_workspace_bytes_dropout(M, N, K, r) >= plain + M * K * 2 + M * K // 8
+    assert q.qlora_workspace_bytes_dropout(0, N, K, r) == 0
