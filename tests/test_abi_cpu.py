@@ -142,3 +142,24 @@ def test_dropout_host_validation_without_gpu(lib):
     plain = q.qlora_workspace_bytes(M, N, K, r)
     assert q.qlora_workspace_bytes_dropout(M, N, K, r) >= plain + M * K * 2 + M * K // 8
     assert q.qlora_workspace_bytes_dropout(0, N, K, r) == 0
+
+
+def test_merge_host_validation_without_gpu(lib):
+    """qlora_merge_adapter refuses a bad output type, r outside [1, 256], a non-finite alpha,
+    NULL or unaligned buffers and oversized shapes before touching any device; an empty weight
+    is a no-op."""
+    P = 1 << 20
+    null = None
+
+    def merge(W=P, N=256, K=256, r=8, alpha=16.0, out=P, dtype=1):
+        return lib.qlora_merge_adapter(_p(W) if W else null, N, K, _p(P), _p(P), r, alpha,
+                                       _p(out) if out else null, dtype, null)
+
+    assert merge(dtype=5) == -1
+    assert merge(r=0) == -1 and merge(r=257) == -1
+    assert merge(alpha=float("inf")) == -1 and merge(alpha=float("nan")) == -1
+    assert merge(W=0) == -1 and merge(out=0) == -1
+    assert merge(W=P + 4) == -2
+    assert merge(K=100) == -2
+    assert merge(N=(1 << 24) + 64) == -2
+    assert merge(W=0, N=0, out=0) == 0
