@@ -20,6 +20,8 @@ Workloads (weights are N x K = out x in, activations are M tokens x K):
                  (nu=4) scaled to std 0.02.
 
 W ~ N(0, 0.02^2) unless stated; X, dY ~ N(0, 1); A ~ N(0, 1/K); B ~ N(0, 0.01^2).
+Test cases may override the weight kind (``zero``: an all-zero weight) and B's
+standard deviation, to make the adapter term dominate the layer.
 """
 from __future__ import annotations
 
@@ -68,6 +70,8 @@ def normal_f32(g: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
 
 def weight(seed: int, layer: int, n_out: int, k_in: int, kind: str = "normal") -> np.ndarray:
     """fp32 frozen weight W (n_out x k_in) of one layer."""
+    if kind == "zero":
+        return np.zeros((n_out, k_in), np.float32)
     g = rng(seed, T_W, layer)
     if kind == "normal":
         return normal_f32(g, (n_out, k_in), WEIGHT_STD)
@@ -91,19 +95,20 @@ def activations(seed: int, layer: int, m: int, k: int, tensor_id: int = T_X) -> 
     return to_bf16_bits(normal_f32(rng(seed, tensor_id, layer), (m, k), 1.0))
 
 
-def lora_pair(seed: int, layer: int, n_out: int, k_in: int, r: int):
-    """bf16 bits of A (r x K, N(0, 1/K)) and B (N x r, N(0, 0.01^2))."""
+def lora_pair(seed: int, layer: int, n_out: int, k_in: int, r: int, b_std: float = 0.01):
+    """bf16 bits of A (r x K, N(0, 1/K)) and B (N x r, N(0, b_std^2), 0.01 by default)."""
     a = to_bf16_bits(normal_f32(rng(seed, T_A, layer), (r, k_in), 1.0 / np.sqrt(k_in)))
-    b = to_bf16_bits(normal_f32(rng(seed, T_B, layer), (n_out, r), 0.01))
+    b = to_bf16_bits(normal_f32(rng(seed, T_B, layer), (n_out, r), b_std))
     return a, b
 
 
 def layer_inputs(name: str, layer: int = 0, M: int | None = None, shape=None, r=None,
-                 alpha=None, seed=None):
+                 alpha=None, seed=None, weights: str | None = None, b_std: float = 0.01):
     """All inputs of one layer of a named workload (numpy, host).
 
     Returns dict(W fp32 NxK, X bf16 MxK, dY bf16 MxN, A bf16 rxK, B bf16 Nxr, alpha, r, M).
-    Overrides (M, shape, r, alpha, seed) give smaller cases with the same recipe.
+    Overrides (M, shape, r, alpha, seed) give smaller cases with the same recipe;
+    ``weights`` replaces the workload's weight kind and ``b_std`` B's standard deviation.
     """
     cfg = WORKLOADS[name]
     seed = cfg["seed"] if seed is None else seed
@@ -113,9 +118,9 @@ def layer_inputs(name: str, layer: int = 0, M: int | None = None, shape=None, r=
         m = m[-1]
     r = cfg["r"] if r is None else r
     alpha = cfg["alpha"] if alpha is None else alpha
-    w = weight(seed, layer, n_out, k_in, cfg["weights"])
+    w = weight(seed, layer, n_out, k_in, cfg["weights"] if weights is None else weights)
     x = activations(seed, layer, m, k_in, T_X)
     dy = activations(seed, layer, m, n_out, T_DY)
-    a, b = lora_pair(seed, layer, n_out, k_in, r)
+    a, b = lora_pair(seed, layer, n_out, k_in, r, b_std)
     return dict(W=w, X=x, dY=dy, A=a, B=b, alpha=float(alpha), r=int(r), M=int(m),
                 N=int(n_out), K=int(k_in))

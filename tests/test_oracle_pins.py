@@ -579,6 +579,108 @@ def test_dropout_bwd_against_finite_differences():
             assert abs(num - grad[idx]) <= 1e-6 * max(1.0, abs(num)), (name, idx, num, grad[idx])
 
 
+def test_dropout_hand_case_at_p_half():
+    """Two tokens, K = N = 2, r = 1, alpha = 1 (s = 1), p = 0.5 (1/(1-p) = 2) and a fixed mask,
+    worked by hand from the PEFT LoRA layer (dropout on the adapter input only):
+    Xd = 2 X*keep = [[2, 0], [0, -2]], U = Xd A^T = [2, -2], X W^T = [[-1, 4], [5, 1]],
+    s U B^T = [[8, -2], [-8, 2]]; V = dY B = [4, -1], dY W = [[2, -1], [1, 1]],
+    2 (V A)*keep = [[8, 0], [0, -2]], dA = s V^T Xd = [8, 2], dB = s dY^T U = [2, -2].
+    A missing or inverted 1/(1-p), a mask on the frozen path, or an unmasked dX adapter term
+    each change these numbers."""
+    X = np.array([[1.0, 3.0], [2.0, -1.0]])
+    keep = np.array([[1, 0], [0, 1]], np.uint8)
+    W = np.array([[2.0, -1.0], [1.0, 1.0]])
+    A = np.array([[1.0, 1.0]])
+    B = np.array([[4.0], [-1.0]])
+    dY = np.array([[1.0, 0.0], [0.0, 1.0]])
+    Y, U = oracle.linear_fwd_dropout(X, W, A, B, 1.0, keep, 0.5)
+    assert np.array_equal(U, [[2.0], [-2.0]])
+    assert np.array_equal(Y, [[7.0, 2.0], [-3.0, 3.0]])
+    dX, dA, dB = oracle.linear_bwd_dropout(X, W, A, B, dY, 1.0, keep, 0.5)
+    assert np.array_equal(dX, [[10.0, -1.0], [1.0, -1.0]])
+    assert np.array_equal(dA, [[8.0, 2.0]])
+    assert np.array_equal(dB, [[2.0], [-2.0]])
+
+
+def test_dropout_exact_rational_case_at_p_half():
+    """Dyadic inputs and a Philox mask at p = 0.5: every product and sum is exact in fp64, so
+    the oracle must equal exact rational arithmetic of Y = X W^T + s (2 X*keep) A^T B^T and of
+    its gradients, written element by element."""
+    g = np.random.default_rng(11)
+    M, N, K, r, alpha = 3, 4, 64, 2, 6.0
+    X = g.integers(-8, 9, (M, K)) / 4.0
+    W = g.integers(-8, 9, (N, K)) / 8.0
+    A = g.integers(-4, 5, (r, K)) / 16.0
+    B = g.integers(-4, 5, (N, r)) / 2.0
+    dY = g.integers(-4, 5, (M, N)) / 2.0
+    keep = oracle.dropout_keep(M, K, 0.5, seed=5, offset=1)
+    assert 0 < keep.sum() < keep.size
+    F = Fraction
+    s = F(alpha) / r
+    Xd = [[F(X[m, k]) * keep[m, k] * 2 for k in range(K)] for m in range(M)]
+    U = [[sum(Xd[m][k] * F(A[j, k]) for k in range(K)) for j in range(r)] for m in range(M)]
+    V = [[sum(F(dY[m, n]) * F(B[n, j]) for n in range(N)) for j in range(r)] for m in range(M)]
+    Yq = [[sum(F(X[m, k]) * F(W[n, k]) for k in range(K)) + s * sum(U[m][j] * F(B[n, j]) for j in range(r))
+           for n in range(N)] for m in range(M)]
+    dXq = [[sum(F(dY[m, n]) * F(W[n, k]) for n in range(N))
+            + s * sum(V[m][j] * F(A[j, k]) for j in range(r)) * keep[m, k] * 2 for k in range(K)] for m in range(M)]
+    dAq = [[s * sum(V[m][j] * Xd[m][k] for m in range(M)) for k in range(K)] for j in range(r)]
+    dBq = [[s * sum(F(dY[m, n]) * U[m][j] for m in range(M)) for j in range(r)] for n in range(N)]
+    Y, Uo = oracle.linear_fwd_dropout(X, W, A, B, alpha, keep, 0.5)
+    dX, dA, dB = oracle.linear_bwd_dropout(X, W, A, B, dY, alpha, keep, 0.5)
+    for got, want in ((Y, Yq), (Uo, U), (dX, dXq), (dA, dAq), (dB, dBq)):
+        assert [[F(v) for v in row] for row in got.tolist()] == want
+
+
+def test_dropout_leaves_the_frozen_path_unmasked():
+    """B = 0 removes the adapter from Y, and A = 0 removes it from dX: whatever the mask, the
+    frozen product X W^T (and dY W) must come out unmasked and unscaled (numpy matmul)."""
+    X, W, A, B, dY = _small_case(M=6, N=10, K=64, r=3, seed=8)
+    for p in (0.3, 0.5, 0.9):
+        keep = oracle.dropout_keep(6, 64, p, seed=3, offset=2)
+        assert keep.sum() < keep.size
+        Y, U = oracle.linear_fwd_dropout(X, W, A, np.zeros_like(B), 4.0, keep, p)
+        assert np.allclose(Y, X @ W.T, rtol=1e-13, atol=1e-13)
+        dX, _, _ = oracle.linear_bwd_dropout(X, W, np.zeros_like(A), B, dY, 4.0, keep, p)
+        assert np.allclose(dX, dY @ W, rtol=1e-13, atol=1e-13)
+
+
+def _nearest_f32(q: Fraction) -> float:
+    """Exact rational -> nearest fp32 (ties to even), for positive normal values."""
+    e = math.floor(math.log2(q))
+    while Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    scaled = q / Fraction(2) ** (e - 23)          # in [2^23, 2^24)
+    m = math.floor(scaled)
+    rem = scaled - m
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and m % 2 == 1):
+        m += 1
+    return float(np.float32(m * 2.0 ** (e - 23)))
+
+
+def test_dropout_scale_on_its_own():
+    """The kept-input scale is 1/(1 - p) of the fp32 p, rounded once to fp32 (exact rational
+    check), and it makes the masked input unbiased: the mean of X*keep*scale over 2^20 ones is
+    1 within the binomial bound (a (1 - p) factor, or none, would miss by p or more)."""
+    for p in (0.05, 0.1, 0.3, 0.5, 0.75, 0.999):
+        p32 = Fraction(float(np.float32(p)))
+        assert oracle.dropout_scale(p) == _nearest_f32(1 / (1 - p32)), p
+    assert oracle.dropout_scale(0.5) == 2.0 and oracle.dropout_scale(0.75) == 4.0
+    for p in (0.05, 0.5):
+        keep = oracle.dropout_keep(1024, 1024, p, seed=21, offset=0)
+        n = keep.size
+        mean = float(keep.mean()) * oracle.dropout_scale(p)
+        keep_rate = 1 - oracle.dropout_threshold(p) / 65536.0
+        assert abs(mean - keep_rate * oracle.dropout_scale(p)) <= 5 * np.sqrt(p * (1 - p) / n) * oracle.dropout_scale(p)
+        assert abs(mean - 1.0) <= 5 * np.sqrt(p * (1 - p) / n) * oracle.dropout_scale(p) + 2.0 ** -15
+        X = np.ones((4, 64))
+        Y, U = oracle.linear_fwd_dropout(X, np.zeros((1, 64)), np.ones((1, 64)), np.zeros((1, 1)), 1.0,
+                                         keep[:4, :64], p)
+        assert np.allclose(U[:, 0], keep[:4, :64].sum(axis=1) * oracle.dropout_scale(p), rtol=1e-15)
+
+
 # ----------------------------------------------------------------- linear
 def _small_case(M=9, N=24, K=64, r=3, seed=0):
     g = np.random.default_rng(seed)

@@ -168,6 +168,72 @@ def test_all_fp32_near_every_threshold_exact():
     check_exact(W.reshape(1, -1), dequant=False)
 
 
+def _threshold_probe_weight(absmax_values: np.ndarray, half_width: int) -> np.ndarray:
+    """Blocks whose absmax is each given value a, holding every fp32 w within half_width ulps
+    of fp32(mid_i * a) for each of the 15 exact midpoints mid_i between neighbouring levels:
+    fp32(w / a) then walks across every decision threshold one ulp at a time, on both sides
+    of the fast path's guard band, with a reciprocal of a that is not exact."""
+    _, t32 = oracle.nf4_codebook()
+    mids = (t32[:-1].astype(np.float64) + t32[1:].astype(np.float64)) / 2
+    offs = np.arange(-half_width, half_width, dtype=np.int64)
+    rows = []
+    for j, a in enumerate(absmax_values.astype(np.float32)):
+        c = (mids * np.float64(a)).astype(np.float32)
+        cb = c.view(np.uint32).astype(np.int64)
+        probes = (cb[:, None] + offs[None, :]).astype(np.uint32).view(np.float32).reshape(-1)
+        assert np.all(np.abs(probes) < a)
+        nb = (probes.size + 62) // 63
+        blk = np.zeros((nb, 64), np.float32)
+        flat = np.zeros(nb * 63, np.float32)
+        flat[:probes.size] = probes
+        blk[:, :63] = flat.reshape(nb, 63)
+        blk[:, 63] = a if j % 2 == 0 else -a          # the block's absmax, either sign
+        rows.append(blk.reshape(-1))
+    return np.concatenate(rows).reshape(1, -1)
+
+
+def test_thresholds_under_inexact_reciprocals_exact():
+    """~1000 block absmax values that are not powers of two, across binades from 2^-100 to
+    2^100 and at both ends of a binade's mantissa range, each with every fp32 weight within
+    2^12 ulps of the 15 scaled thresholds: the fast reciprocal path and its guard must give
+    the codes of one IEEE division, bit for bit."""
+    g = np.random.default_rng(2024)
+    mant = g.uniform(1.0, 2.0, 960)
+    expo = g.integers(-100, 101, 960)
+    vals = [np.float32(m * 2.0 ** e) for m, e in zip(mant, expo)]
+    for e in (-20, -7, -1, 0, 3):
+        for m in (1.0 + 2.0 ** -23, 1.0 + 2.0 ** -22, 1.5, 2.0 - 2.0 ** -23, 2.0 - 2.0 ** -21):
+            vals.append(np.float32(m * 2.0 ** e))
+    vals += [np.float32(0.0173), np.float32(3 * 2.0 ** -20), np.float32(0.0731), np.float32(3.3e-3)]
+    a = np.array(vals, np.float32)
+    assert not np.any(np.frexp(a)[0] == 0.5)          # no power of two among them
+    for part in np.array_split(a, 4):
+        check_exact(_threshold_probe_weight(part, 1 << 12), dequant=False)
+    check_exact(_threshold_probe_weight(a[::40], 1 << 8), dequant=True)
+
+
+def test_every_fp32_in_unit_interval_exact():
+    """Every fp32 n in [-1, 1] (2,130,706,434 values, zeros of both signs included), 63 to a
+    block with -1.0 as the block's absmax so that w / absmax = n exactly: the GPU's codes equal
+    the oracle's exact nearest-level rule on all of them.  Streamed in chunks of 2^26 weights."""
+    per_chunk = (1 << 26) // 64                           # blocks per chunk
+    pos = np.arange(0, 0x3F800001, dtype=np.int64)       # +0.0 .. 1.0
+    total = 2 * pos.size
+    done = 0
+    while done < total:
+        k = min(per_chunk * 63, total - done)
+        idx = np.arange(done, done + k, dtype=np.int64)
+        bits = np.where(idx < pos.size, idx, (idx - pos.size) | 0x80000000).astype(np.uint32)
+        nb = (k + 62) // 63
+        flat = np.zeros(nb * 63, np.float32)
+        flat[:k] = bits.view(np.float32)
+        W = np.empty((nb, 64), np.float32)
+        W[:, :63] = flat.reshape(nb, 63)
+        W[:, 63] = -1.0
+        check_exact(W.reshape(1, -1), dequant=False)
+        done += k
+
+
 def test_random_fp32_in_unit_interval_exact():
     g = np.random.default_rng(123)
     bits = g.integers(0, 0x3F800001, size=(1 << 22), dtype=np.uint32)
