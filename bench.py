@@ -670,23 +670,23 @@ def run_ours(args, rank, world, local_rank):
 
     if args.profile:
         # profiling case for ncu: one step to load the modules, one step to
-        # capture, then two decode forwards (M = 1, r = 8) on the same weight.
-        # Launches: [L2 flush write + L2 flush read + 6 step kernels] x 2, then
-        # 2 decode kernels.
+        # capture, then decode forwards (r = 8) on the same weight: two at
+        # M = 1, then two at M = 16.  Launches: [L2 flush write + L2 flush read
+        # + 6 step kernels] x 2, then 4 decode kernels.
         from bit_nf4_quantized_quantize_b200 import synth
-        dinp = synth.layer_inputs("decode", M=1)
-        decX, decA, decB = (torch.from_numpy(dinp[k].view(np.int16)).view(torch.bfloat16).to(dev)
-                            for k in ("X", "A", "B"))
-        decY = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
-        dws = torch.empty(q.qlora_workspace_bytes(1, N, K, DECODE_RANK), dtype=torch.uint8, device=dev)
+        dinp = synth.layer_inputs("decode", M=16)
+        decA, decB = (torch.from_numpy(dinp[k].view(np.int16)).view(torch.bfloat16).to(dev) for k in ("A", "B"))
         for i in range(2):
             flush(float(i))
             step()
-        for _ in range(2):
+        for dm in (1, 1, 16, 16):
+            decX = torch.from_numpy(dinp["X"][:dm].view(np.int16)).view(torch.bfloat16).to(dev)
+            decY = torch.empty(dm, N, dtype=torch.bfloat16, device=dev)
+            dws = torch.empty(q.qlora_workspace_bytes(dm, N, K, DECODE_RANK), dtype=torch.uint8, device=dev)
             q.qlora_linear_fwd(codes, q8, s2, N, K, decX, decA, decB, dinp["alpha"], Y=decY, workspace=dws)
         torch.cuda.synchronize()
         rc = q.qlora_device_status()
-        print(json.dumps({"profile_case": WORKLOAD + " step + decode M=1", "device_status": rc}), flush=True)
+        print(json.dumps({"profile_case": WORKLOAD + " step + decode M=1, M=16", "device_status": rc}), flush=True)
         if rc != 0:
             raise RuntimeError(q.qlora_strerror(rc))
         return

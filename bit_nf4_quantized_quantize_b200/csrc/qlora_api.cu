@@ -1193,13 +1193,15 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
       }
       gst = aux->s;
     }
-    if (int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, gst, dev,
-                                         QLORA_KERNEL_GRAD_GEMM, unsplit ? 2 : 1))
-      return rc;
+    const int rc = launch_lora<true, true>(ta0, tb0, ta1, tb1, la, tiles_a + tiles_b, S, gst, dev,
+                                           QLORA_KERNEL_GRAD_GEMM, unsplit ? 2 : 1);
+    // the second stream joins back even when the launch failed, so that a capture on the
+    // caller's stream never ends with an unjoined branch
     if (aux && (cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)) {
       cudaGetLastError();
-      return QLORA_ERR_CUDA;
+      return rc ? rc : QLORA_ERR_CUDA;
     }
+    if (rc) return rc;
   }
   return QLORA_OK;
 }

@@ -65,7 +65,18 @@ constexpr int kLutCells = 33;  // floor(16 n) + 16 for n in [-1, 1]
 constexpr int kLutPad = 64;    // table entries in shared memory: any 6-bit index is in range
 constexpr float kCellOffset = 15.875f;     // t = 16 n + 15.875
 constexpr float kQuarterMagic = 3145728.f;  // 1.5 * 2^21: fp32 values in [2^21, 2^22) have ulp 1/4
-constexpr float kFastGuard = 6.103515625e-05f;  // 2^-14, in units of t
+// Guard of the fast path, in units of t.  With n = fp32(w / absmax), |w / absmax| <= 1,
+// and the exact decision "n > mid" read as 16 n + 15.875 > T, T = 16 mid + 15.875:
+//   |t' - (16 w/absmax + 15.875)| <= 16 * 2^-23 (rcp.approx, relative error <= 2^-23)
+//                                    + 2^-20 (the fma's rounding: t' < 32, ulp <= 2^-19)
+//   |16 n - 16 w/absmax|          <= 16 * 2^-25 = 2^-21 (the rounding of n)
+//   so |t' - (16 n + 15.875)|     <  2^-18;
+//   |B - T| <= 2^-20 (rounding T to fp32) + 15 * 2^-19 (the code in the 4 low mantissa
+//   bits)  <  2^-15.
+// If |B - t'| > 2^-14 > 2^-15 + 2^-18, B - t' and T - (16 n + 15.875) have the same sign, so
+// the fast code is the exact one; the margin is about 1.8x.  fabsf(B - t') is exact where it
+// is near 2^-14 (B and t' within a factor 2 of each other), so the test itself cannot err.
+constexpr float kFastGuard = 6.103515625e-05f;  // 2^-14
 
 // Host-built tables handed to the kernels by value.
 struct Nf4Tables {

@@ -223,7 +223,9 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
  *   as long as launch timing (qlora_timing_enable) is off, which is the default.
  * - Set-up: the first call on a device looks up the scratch's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it.  Make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  The cached address belongs to the
+ *   device's primary context: after cudaDeviceReset it is stale, so do not
+ *   call this entry point again in that process.
  * - Sharing: every call uses the same scratch, which keeps the last call's
  *   contents.  Every element this path reads is written by the same call first,
  *   so nothing needs clearing.  Calls that overlap on the GPU (different
