@@ -328,38 +328,55 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       // (now idle) stage memory and written by one TMA bulk tensor store,
       // which also clips rows >= M and columns >= N.
       uint8_t* stage = smem + (warp - 2) * (MH * 4 * 2048);
-#pragma unroll 1
-      for (int h = 0; h < MH; ++h) {
-        uint32_t v[4][32];
-        const uint32_t tbase = tmem_d + (static_cast<uint32_t>(q * 32) << 16) + h * kPairN;
+      // The warp's 4 * MH chunks of 32 columns, c = 4 h + j at half h, column chunk wg + 2 j.
+      // Two register buffers: the load of chunk c + 1 is in flight while chunk c is
+      // converted and staged; the wait that follows hands its registers over.
+      constexpr int kChunks = 4 * MH;
+      const uint32_t tlane = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+      auto chunk_col = [&](int c) -> uint32_t {
+        return static_cast<uint32_t>((c >> 2) * kPairN + (wg + 2 * (c & 3)) * 32);
+      };
+      auto stage_chunk = [&](int c, const uint32_t (&v)[32]) {
+        // row `lane` of the block: 64 bytes, 16-byte chunk i at (i ^ ((lane >> 1) & 3))
+        const uint32_t blk = smem_u32(stage + c * 2048);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld_32x32b_x32(tbase + (wg + 2 * j) * 32, v[j]);
-        tmem_ld_wait();
+        for (int i = 0; i < 4; ++i) {
+          uint4 o;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+          o.x = *reinterpret_cast<uint32_t*>(&h0);
+          o.y = *reinterpret_cast<uint32_t*>(&h1);
+          o.z = *reinterpret_cast<uint32_t*>(&h2);
+          o.w = *reinterpret_cast<uint32_t*>(&h3);
+          st_shared_v4(blk + lane * 64 + ((static_cast<uint32_t>(i) ^ ((lane >> 1) & 3)) << 4), o);
+        }
+        if ((c & 3) == 3) {
+          // the half's four blocks are staged: store them
+          const int h = c >> 2;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int row0 = m0 + 256 * h + 128 * static_cast<int>(rank) + q * 32;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // row `lane` of the block: 64 bytes, 16-byte chunk c at (c ^ ((lane >> 1) & 3))
-          const uint32_t blk = smem_u32(stage + (h * 4 + j) * 2048);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 o;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 0]), __uint_as_float(v[j][8 * i + 1]));
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 2]), __uint_as_float(v[j][8 * i + 3]));
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 4]), __uint_as_float(v[j][8 * i + 5]));
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[j][8 * i + 6]), __uint_as_float(v[j][8 * i + 7]));
-            o.x = *reinterpret_cast<uint32_t*>(&h0);
-            o.y = *reinterpret_cast<uint32_t*>(&h1);
-            o.z = *reinterpret_cast<uint32_t*>(&h2);
-            o.w = *reinterpret_cast<uint32_t*>(&h3);
-            st_shared_v4(blk + lane * 64 + ((static_cast<uint32_t>(i) ^ ((lane >> 1) & 3)) << 4), o);
+            for (int j = 0; j < 4; ++j)
+              tma_store_2d(&tmOut, stage + (h * 4 + j) * 2048, c0 + (wg + 2 * j) * 32, row0);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int row0 = m0 + 256 * h + 128 * static_cast<int>(rank) + q * 32;
+      };
+      uint32_t va[32], vb[32];
+      tmem_ld_32x32b_x32(tlane + chunk_col(0), va);
+      tmem_ld_wait_regs(va);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_store_2d(&tmOut, stage + (h * 4 + j) * 2048, c0 + (wg + 2 * j) * 32, row0);
+      for (int c = 0; c < kChunks; c += 2) {
+        if (c + 1 < kChunks) tmem_ld_32x32b_x32(tlane + chunk_col(c + 1), vb);
+        stage_chunk(c, va);
+        if (c + 1 < kChunks) {
+          tmem_ld_wait_regs(vb);
+          if (c + 2 < kChunks) tmem_ld_32x32b_x32(tlane + chunk_col(c + 2), va);
+          stage_chunk(c + 1, vb);
+          if (c + 2 < kChunks) tmem_ld_wait_regs(va);
         }
       }
       if (lane == 0) {
