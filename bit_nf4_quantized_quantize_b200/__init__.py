@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     exported_symbols,
     lib_path,
     load,
+    qlora_debug_record,
     qlora_dequant,
     qlora_dropout_apply,
     qlora_launch_count,

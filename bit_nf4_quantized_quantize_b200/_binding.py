@@ -4,6 +4,10 @@ Each function checks tensor dtypes/devices/contiguity, allocates outputs the
 caller did not pass (torch device memory), and calls the C entry point with
 raw device pointers and torch's current stream.  Non-zero return codes raise
 QloraError.
+
+With QLORA_CHECKED_LIBRARY=1 in the environment the binding loads the checked
+build, libqlora_nf4_debug.so (bounds and alignment checks before every TMA
+copy and cluster exchange; qlora_debug_record reads what they found).
 """
 from __future__ import annotations
 
@@ -14,7 +18,8 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+_LIB_PATH = os.path.join(_HERE, "libqlora_nf4_debug.so" if os.environ.get("QLORA_CHECKED_LIBRARY") == "1"
+                         else "libqlora_nf4.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -68,6 +73,7 @@ _SIGNATURES = {
     "qlora_timing_enable": (ctypes.c_int, [ctypes.c_int]),
     "qlora_timing_collect": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]),
     "qlora_launch_count": (ctypes.c_int64, []),
+    "qlora_debug_record": (ctypes.c_int, [ctypes.c_void_p]),
 }
 
 KERNEL_KINDS = ["quantize", "dequant", "lora_gemm", "lora_reduce", "fwd_fused", "dx_fused", "grad_gemm",
@@ -432,6 +438,14 @@ def qlora_timing_collect() -> dict:
     _check(load().qlora_timing_collect(ms.ctypes.data_as(ctypes.c_void_p), cnt.ctypes.data_as(ctypes.c_void_p),
                                        len(KERNEL_KINDS)), "qlora_timing_collect")
     return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS) if cnt[i]}
+
+
+def qlora_debug_record() -> dict:
+    """Read and clear the checked build's record of failed checks (current device):
+    {failed, first_code, first_value, first_cta}.  The ordinary build raises QloraError."""
+    out = (ctypes.c_int64 * 4)()
+    _check(load().qlora_debug_record(ctypes.byref(out)), "qlora_debug_record")
+    return {"failed": int(out[0]), "first_code": int(out[1]), "first_value": int(out[2]), "first_cta": int(out[3])}
 
 
 def qlora_launch_count() -> int:

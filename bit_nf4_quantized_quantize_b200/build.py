@@ -3,6 +3,10 @@
 The library is one translation unit (csrc/qlora_api.cu includes the kernel
 headers), compiled with IEEE division and denormal support (no fast math):
 the quantizer's codes depend on correctly rounded fp32 division.
+
+`--debug` builds the checked library (libqlora_nf4_debug.so, QLORA_DEBUG):
+the same kernels with bounds and alignment checks before every TMA copy and
+cluster exchange (include/qlora_nf4.h, qlora_debug_record).
 """
 from __future__ import annotations
 
@@ -15,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlora_nf4.so")
+LIB_DEBUG = os.path.join(PKG, "libqlora_nf4_debug.so")
 SOURCES = [os.path.join(CSRC, "qlora_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "qlora_nf4.h")]
@@ -32,25 +37,27 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(d) > t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *(extra or []), "-o", tmp, *SOURCES]
+def build(force: bool = False, verbose: bool = False, extra=None, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not needs_build(lib):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    flags = NVCC_FLAGS + (["-DQLORA_DEBUG"] if debug else [])
+    cmd = [nvcc(), *flags, "-I", INCLUDE, "-I", CSRC, *(extra or []), "-o", tmp, *SOURCES]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
+    build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)

@@ -226,7 +226,7 @@ qlora_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         uint8_t* st = smem + s * L::kStageBytes;
         mbar_arrive_expect_tx(&full_tma[s], MP * 128 + T * 32 + r * 128);
         tma_load_2d(st + L::kXOff, &tmX, &full_tma[s], ks * 64, 0);
-        tma_load_2d(st + L::kPOff, &tmP, &full_tma[s], ks * 32, c0);
+        tma_load_2d(st + L::kPOff, &tmP, &full_tma[s], ks * 32, c0, 1);
         tma_load_2d(st + a_off, &tmA, &full_tma[s], ks * 64, 0);
       }
     }
@@ -377,7 +377,9 @@ qlora_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
         for (int m = 0; m < MP; ++m) {
           if (m >= mv) break;
-          const uint32_t off = base + static_cast<uint32_t>(((rank * MP + m) * su_n + jl) * 4);
+          const int uidx = (rank * MP + m) * su_n + jl;
+          if (!QLORA_CHECK(uidx < MP * 72 && o < S, kDbgCluster, uidx)) continue;
+          const uint32_t off = base + static_cast<uint32_t>(uidx * 4);
           if (clustered) st_async_f32(map_to_rank(off, o), u[m], map_to_rank(recv_bar, o));
           else *reinterpret_cast<float*>(smem + L::kRecvUOff + (off - base)) = u[m];
         }
@@ -404,7 +406,9 @@ qlora_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
         for (int m = 0; m < MP; ++m) {
           if (m >= mv) break;
-          const uint32_t off = base + static_cast<uint32_t>(((rank * MP + m) * sl + il) * 4);
+          const int yidx = (rank * MP + m) * sl + il;
+          if (!QLORA_CHECK(yidx < MP * 192 && o < S, kDbgCluster, yidx)) continue;
+          const uint32_t off = base + static_cast<uint32_t>(yidx * 4);
           if (clustered) st_async_f32(map_to_rank(off, o), v[m], map_to_rank(recv_bar, o));
           else *reinterpret_cast<float*>(smem + L::kRecvOff + (off - base)) = v[m];
         }

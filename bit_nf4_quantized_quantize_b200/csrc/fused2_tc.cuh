@@ -217,8 +217,8 @@ qlora_fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
           for (int h = 0; h < MH; ++h)
             tma_load_2d(a_dst + h * kAHalfBytes, &tmA, &full_tma[s], ks * kBK, m0 + 256 * h + 128 * rank);
           uint8_t* p_dst = smem + L::kPOff + s * L::kPTile;
-          if (!kBMN) tma_load_2d(p_dst, &tmP, &full_tma[s], ks * (kBK / 2), cb);   // 128 rows x 32 B
-          else tma_load_2d(p_dst, &tmP, &full_tma[s], cb / 2, ks * kBK);           // 64 rows x 64 B
+          if (!kBMN) tma_load_2d(p_dst, &tmP, &full_tma[s], ks * (kBK / 2), cb, 1);   // 128 rows x 32 B
+          else tma_load_2d(p_dst, &tmP, &full_tma[s], cb / 2, ks * kBK, 1);        // 64 rows x 64 B
         }
       }
     }

@@ -271,10 +271,10 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
               tma_load_2d(b_dst + c * (kBK * 128), &tmB, &full_tma[s], c0 + 64 * c, ks * kBK);
           } else if (BSRC == kBDeqK) {
             // packed codes of weight rows [c0, c0+BN), k-step ks: BN rows x 32 B
-            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], ks * (kBK / 2), c0);
+            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], ks * (kBK / 2), c0, 1);
           } else {
             // packed codes of weight rows [64 ks, 64 ks + 64), columns [c0, c0+BN): 64 rows x BN/2 B
-            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], c0 / 2, ks * kBK);
+            tma_load_2d(smem + L::kPOff + s * L::kPTileBytes, &tmB, &full_tma[s], c0 / 2, ks * kBK, 1);
           }
         }
       }
@@ -562,6 +562,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int row = idx / (BN / 4);
         const int c4 = idx - row * (BN / 4);
         const uint32_t off = static_cast<uint32_t>(row * BN + ((c4 + row) & (BN / 4 - 1)) * 4) * 4u;
+        if (!QLORA_CHECK(off + 16u <= static_cast<uint32_t>(kBM * BN * 4), kDbgCluster, off)) continue;
         float4 v[8];
 #pragma unroll
         for (int p = 0; p < 8; ++p)

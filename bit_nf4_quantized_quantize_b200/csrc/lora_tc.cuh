@@ -232,6 +232,7 @@ qlora_lora_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constan
       }
       const int trow = rank * rows_here + lr;
       const uint32_t off = static_cast<uint32_t>(trow * 64 + ((c16 + trow) & 15) * 4) * 4u;
+      if (!QLORA_CHECK(off + 16u <= 128u * 64u * 4u, kDbgCluster, off)) continue;
       // issue all remote loads before the first add, then sum in rank order
       float4 v[8];
 #pragma unroll

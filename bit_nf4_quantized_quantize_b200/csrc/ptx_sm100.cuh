@@ -22,6 +22,35 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- checked build
+// Built with -DQLORA_DEBUG (libqlora_nf4_debug.so, build.py --debug), every
+// TMA copy checks its coordinates and shared-memory address and every cluster
+// exchange checks its offset before the access.  A failed check is counted in
+// g_debug_record (the first one's code, value and CTA are kept) and the access
+// is skipped, so a wrong index never reaches the memory system: the kernel
+// finishes, its waits ending by their time limit where bytes were skipped.
+// qlora_debug_record reads and clears the record.  Without QLORA_DEBUG the
+// checks compile to nothing.
+constexpr uint32_t kDbgTmaX = 1;        // TMA x coordinate not a multiple of 16 bytes
+constexpr uint32_t kDbgTmaStore = 2;    // TMA store at a negative coordinate
+constexpr uint32_t kDbgSmemAlign = 3;   // shared-memory operand of a copy not 16-byte aligned
+constexpr uint32_t kDbgCluster = 4;     // cluster-exchange offset outside its region
+constexpr uint32_t kDbgBulk = 5;        // bulk copy: address or size not a multiple of 16 bytes
+#ifdef QLORA_DEBUG
+__device__ unsigned long long g_debug_record[4];   // failed checks, first code, first value, first CTA
+__device__ __forceinline__ bool debug_ok(bool ok, uint32_t code, long long value) {
+  if (!ok && atomicAdd(&g_debug_record[0], 1ull) == 0ull) {
+    g_debug_record[1] = code;
+    g_debug_record[2] = static_cast<unsigned long long>(value);
+    g_debug_record[3] = blockIdx.x + static_cast<unsigned long long>(gridDim.x) * (blockIdx.y + gridDim.y * blockIdx.z);
+  }
+  return ok;
+}
+#define QLORA_CHECK(cond, code, value) ::qlora::debug_ok((cond), (code), static_cast<long long>(value))
+#else
+#define QLORA_CHECK(cond, code, value) true
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -114,8 +143,12 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 
 // 2-D tiled bulk tensor load into this CTA's shared memory; completion is
 // signalled as transaction bytes on `bar`.  x is the innermost coordinate.
+// x_bytes: bytes per element of the map (the checked build tests x * x_bytes % 16 == 0).
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y) {
+                                            int32_t x, int32_t y, int32_t x_bytes = 2) {
+  if (!QLORA_CHECK((x * x_bytes) % 16 == 0, kDbgTmaX, x) ||
+      !QLORA_CHECK((smem_u32(smem_dst) & 15u) == 0, kDbgSmemAlign, smem_u32(smem_dst)))
+    return;
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
@@ -126,6 +159,9 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 // 2-D tiled bulk tensor store from this CTA's shared memory (bulk-group
 // completion).  Rows or columns past the tensor's extent are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  if (!QLORA_CHECK(x >= 0 && y >= 0, kDbgTmaStore, x < 0 ? x : y) || !QLORA_CHECK(x % 8 == 0, kDbgTmaX, x) ||
+      !QLORA_CHECK((smem_u32(smem_src) & 15u) == 0, kDbgSmemAlign, smem_u32(smem_src)))
+    return;
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
                ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y) : "memory");
 }

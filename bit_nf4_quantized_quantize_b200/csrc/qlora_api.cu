@@ -770,8 +770,29 @@ const char* qlora_strerror(int code) {
     case QLORA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
     case QLORA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case QLORA_ERR_UNAVAILABLE: return "available in the checked build (libqlora_nf4_debug.so) only";
     default: return "unknown error code";
   }
+}
+
+int qlora_debug_record(int64_t* out) {
+#ifdef QLORA_DEBUG
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  int dev, sms;
+  if (int rc = check_device(&dev, &sms)) return rc;
+  unsigned long long h[4];
+  const unsigned long long zero[4] = {0ull, 0ull, 0ull, 0ull};
+  if (cudaMemcpyFromSymbol(h, qlora::g_debug_record, sizeof(h)) != cudaSuccess ||
+      cudaMemcpyToSymbol(qlora::g_debug_record, zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  for (int i = 0; i < 4; ++i) out[i] = static_cast<int64_t>(h[i]);
+  return QLORA_OK;
+#else
+  (void)out;
+  return QLORA_ERR_UNAVAILABLE;
+#endif
 }
 
 int qlora_nf4_codebook(float* out) {

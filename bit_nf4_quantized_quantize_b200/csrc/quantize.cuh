@@ -215,6 +215,10 @@ quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, int64_t group
   };
   auto issue = [&](int64_t g, int s) {
     const uint32_t bytes = static_cast<uint32_t>(group_blocks(g)) * kBlock * 4u;
+    if (!QLORA_CHECK((bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(W + g * kGroupFloats) & 15u) == 0 &&
+                         (smem_u32(sm.stage[s]) & 15u) == 0,
+                     kDbgBulk, bytes))
+      return;
     ++sm.issued[s];
     mbar_arrive_expect_tx(&sm.full[s], bytes);
     bulk_load_g2s(sm.stage[s], W + g * kGroupFloats, bytes, &sm.full[s]);

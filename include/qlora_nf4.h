@@ -83,6 +83,7 @@ extern "C" {
 #define QLORA_ERR_DEVICE_TIMEOUT (-4)  /* a kernel's bounded wait expired           */
 #define QLORA_ERR_WORKSPACE (-5)       /* workspace NULL or smaller than required   */
 #define QLORA_ERR_NO_DEVICE (-6)       /* no sm_100 device is current               */
+#define QLORA_ERR_UNAVAILABLE (-7)     /* the call needs the checked build           */
 
 #define QLORA_OUT_BF16 0
 #define QLORA_OUT_FP32 1
@@ -361,6 +362,27 @@ int qlora_timing_enable(int on);
  * devices, all streams), counted whether or not timing is enabled. */
 int64_t qlora_launch_count(void);
 int qlora_timing_collect(double* ms, int64_t* counts, int n_kinds);
+
+/*
+ * Checked build: libqlora_nf4_debug.so, the same library compiled with
+ * QLORA_DEBUG (build.py --debug).  Its kernels check, before each access, the
+ * coordinates and shared-memory address of every TMA copy (x a multiple of 16
+ * bytes, no store at a negative coordinate, 16-byte aligned shared memory), the
+ * offsets of every cluster exchange (inside the receiving region) and the
+ * alignment of the quantizer's bulk copies.  A failed check is counted, the
+ * first one's code, value and CTA are kept, and the access is skipped (the
+ * kernel then ends through its bounded waits, with QLORA_ERR_DEVICE_TIMEOUT).
+ * It stands in for a memory checker on GPUs where none can run; results are
+ * bit-identical to the ordinary build's.  No counterpart on the pages.
+ *
+ *   out[0] failed checks since the last call, out[1] the first one's code
+ *   (1 TMA x misaligned, 2 TMA store at a negative coordinate, 3 shared-memory
+ *   address misaligned, 4 cluster-exchange offset out of range, 5 bulk copy
+ *   misaligned), out[2] its value, out[3] its CTA (linear index).  out: host
+ *   int64[4].  Reads and clears the record of the current device; synchronises
+ *   with the device.  The ordinary build returns QLORA_ERR_UNAVAILABLE.
+ */
+int qlora_debug_record(int64_t* out);
 
 #ifdef __cplusplus
 }

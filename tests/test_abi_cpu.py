@@ -42,6 +42,20 @@ def test_every_declared_symbol_is_exported(lib):
     assert declared == set(q._binding._SIGNATURES)
 
 
+def test_checked_build_exports_the_same_symbols(lib):
+    """The checked build (QLORA_DEBUG) compiles for sm_100a and exports every declared
+    symbol; the ordinary build answers qlora_debug_record with QLORA_ERR_UNAVAILABLE
+    without touching a GPU."""
+    path = qbuild.build(debug=True)
+    assert path.endswith("libqlora_nf4_debug.so") and os.path.exists(path)
+    dlib = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(dlib, name), name
+    out = (ctypes.c_int64 * 4)()
+    assert lib.qlora_debug_record(ctypes.byref(out)) == -7
+    assert b"checked build" in lib.qlora_strerror(-7)
+
+
 def test_library_codebook_equals_oracle_bitwise(lib):
     ours = q.qlora_nf4_codebook()
     _, ref = oracle.nf4_codebook()
