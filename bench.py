@@ -587,19 +587,24 @@ def run_dropout(q, dev, peaks, p=0.05, reps=10):
     dA = torch.empty(r, K, dtype=torch.float32, device=dev)
     dB = torch.empty(N, r, dtype=torch.float32, device=dev)
     ws = torch.empty(q.qlora_workspace_bytes_dropout(M, N, K, r), dtype=torch.uint8, device=dev)
+    # the state a training framework keeps for dropout's backward: the masked input and the mask
+    Xd = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    keep = torch.empty(M * K // 32, dtype=torch.int32, device=dev)
     it = [0]
 
     def step():
         it[0] += 1   # a fresh mask every step: offset = step index
-        q.qlora_linear_fwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, 1234, it[0], Y=Y, U_save=U, workspace=ws)
+        q.qlora_linear_fwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, 1234, it[0], Y=Y, U_save=U, Xd_save=Xd,
+                                   keep_save=keep, workspace=ws)
         q.qlora_linear_bwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, 1234, it[0], dY, U_saved=U, dX=dX, dA=dA,
-                                   dB=dB, workspace=ws)
+                                   dB=dB, Xd_saved=Xd, keep_saved=keep, workspace=ws)
 
     ms = time_region(step, 3, reps)
     rc = q.qlora_device_status()
     if rc != 0:
         raise RuntimeError(f"device status after the dropout region: {q.qlora_strerror(rc)}")
-    return {"workload": f"train4096 layer fwd+bwd with LoRA dropout p={p} on the adapter input",
+    return {"workload": f"train4096 layer fwd+bwd with LoRA dropout p={p} on the adapter input; the forward "
+                        "keeps the masked input and the keep bits for the backward",
             "fwd_bwd_ms": ms, "fwd_bwd_tflops": step_flops(M, N, K, r) / (ms * 1e-3) / 1e12}
 
 

@@ -60,11 +60,13 @@ _SIGNATURES = {
                                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                                 ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_linear_bwd_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                                 ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_dropout_apply": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
@@ -362,9 +364,21 @@ def _workspace_dropout(ws, M, N, K, r, device):
     return ws
 
 
+def _dropout_state(Xd, keep, M: int, k_in: int, names):
+    """Validate kept dropout state: bf16 [M, K] masked input and int32 [M*K/32] keep words, both or neither."""
+    if (Xd is None) != (keep is None):
+        raise ValueError(f"{names[0]} and {names[1]} go together")
+    if Xd is not None:
+        _dev(Xd, torch.bfloat16, names[0], (M, k_in))
+        _dev(keep, torch.int32, names[1], (M * k_in // 32,))
+
+
 def qlora_linear_fwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float, p: float, seed: int,
-                             offset: int, Y=None, U_save=None, workspace=None, stream=None):
-    """The forward with dropout p on the adapter input (Philox keep mask from seed, offset)."""
+                             offset: int, Y=None, U_save=None, Xd_save=None, keep_save=None, workspace=None,
+                             stream=None):
+    """The forward with dropout p on the adapter input (Philox keep mask from seed, offset).
+    Xd_save (bf16 [M, K]) and keep_save (int32 [M*K/32]), if given, receive the masked input
+    and the keep bits, for the backward to read instead of generating the mask again."""
     _weight(codes, q8, s2, n_out, k_in)
     M = X.shape[0]
     r = A.shape[0]
@@ -374,18 +388,21 @@ def qlora_linear_fwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
     Y = torch.empty(M, n_out, dtype=torch.bfloat16, device=X.device) if Y is None else _dev(Y, torch.bfloat16, "Y", (M, n_out))
     if U_save is not None:
         _dev(U_save, torch.bfloat16, "U_save", (M, r))
+    _dropout_state(Xd_save, keep_save, M, k_in, ("Xd_save", "keep_save"))
     ws = _workspace_dropout(workspace, M, n_out, k_in, r, X.device)
     _check(load().qlora_linear_fwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
                                            _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(Y),
-                                           _ptr(U_save), _ptr(ws), _nbytes(ws), _stream(stream)),
+                                           _ptr(U_save), _ptr(Xd_save), _ptr(keep_save), _ptr(ws), _nbytes(ws),
+                                           _stream(stream)),
            "qlora_linear_fwd_dropout")
     return Y
 
 
 def qlora_linear_bwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alpha: float, p: float, seed: int,
                              offset: int, dY, U_saved=None, dX=None, dA=None, dB=None, need_dX=True,
-                             workspace=None, stream=None):
-    """The backward with dropout p on the adapter input -> (dX or None, dA, dB)."""
+                             Xd_saved=None, keep_saved=None, workspace=None, stream=None):
+    """The backward with dropout p on the adapter input -> (dX or None, dA, dB).  Xd_saved and
+    keep_saved: the state a forward kept (same p, seed, offset), or None to generate the mask."""
     _weight(codes, q8, s2, n_out, k_in)
     M = X.shape[0]
     r = A.shape[0]
@@ -402,11 +419,12 @@ def qlora_linear_bwd_dropout(codes, q8, s2, n_out: int, k_in: int, X, A, B, alph
         dX = None
     dA = torch.empty(r, k_in, dtype=torch.float32, device=dev) if dA is None else _dev(dA, torch.float32, "dA", (r, k_in))
     dB = torch.empty(n_out, r, dtype=torch.float32, device=dev) if dB is None else _dev(dB, torch.float32, "dB", (n_out, r))
+    _dropout_state(Xd_saved, keep_saved, M, k_in, ("Xd_saved", "keep_saved"))
     ws = _workspace_dropout(workspace, M, n_out, k_in, r, dev)
     _check(load().qlora_linear_bwd_dropout(_ptr(codes), _ptr(q8), _ptr(s2), n_out, k_in, _ptr(X), M, _ptr(A),
                                            _ptr(B), r, float(alpha), float(p), int(seed), int(offset), _ptr(dY),
-                                           _ptr(U_saved), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), _nbytes(ws),
-                                           _stream(stream)),
+                                           _ptr(U_saved), _ptr(Xd_saved), _ptr(keep_saved), _ptr(dX), _ptr(dA),
+                                           _ptr(dB), _ptr(ws), _nbytes(ws), _stream(stream)),
            "qlora_linear_bwd_dropout")
     return dX, dA, dB
 

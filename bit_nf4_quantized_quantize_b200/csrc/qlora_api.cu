@@ -592,6 +592,10 @@ struct DropoutSpec {
   uint32_t t = 0;
   float inv = 1.f;
   uint64_t seed = 0, offset = 0;
+  // the masked input X * keep and the keep bits: written by the forward when the caller
+  // asks to keep them, read by the backward instead of being generated again
+  uint16_t* xd = nullptr;
+  uint16_t* bits = nullptr;
 };
 
 // Returns false if p is not in [0, 1).  p == 0 leaves the spec off.
@@ -945,8 +949,8 @@ static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   const bool beside = M > 128 && adapter_beside(M, rpad, pairs, sms);
   if (dr.on) {
     // the adapter's input goes through dropout: U = (X * keep) A^T / (1 - p)
-    uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
-    if (int rc = launch_dropout_mask(X, M, k_in, dr, Xm, sms, st)) return rc;
+    uint16_t* Xm = dr.xd ? dr.xd : reinterpret_cast<uint16_t*>(ws + L.xm);
+    if (int rc = launch_dropout_mask(X, M, k_in, dr, Xm, sms, st, dr.bits)) return rc;
     if (int rc = run_lora_down(Xm, M, k_in, A, r, dr.inv, s * dr.inv, U_save, Us, sms, st, dev, beside)) return rc;
   } else if (int rc = run_lora_down(X, M, k_in, A, r, 1.f, s, U_save, Us, sms, st, dev, beside)) {
     return rc;
@@ -999,12 +1003,25 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
                   DropoutSpec{});
 }
 
+// The kept dropout state: the masked input and the keep bits, both or neither.
+static int dropout_state(const void* xd, const void* bits, DropoutSpec* dr) {
+  if ((xd == nullptr) != (bits == nullptr)) return QLORA_ERR_INVALID_ARG;
+  if ((xd && !aligned16(xd)) || (bits && !aligned16(bits))) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (dr->on) {
+    dr->xd = const_cast<uint16_t*>(static_cast<const uint16_t*>(xd));
+    dr->bits = const_cast<uint16_t*>(static_cast<const uint16_t*>(bits));
+  }
+  return QLORA_OK;
+}
+
 int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
                              const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
-                             float p, uint64_t seed, uint64_t offset, uint16_t* Y, uint16_t* U_save, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+                             float p, uint64_t seed, uint64_t offset, uint16_t* Y, uint16_t* U_save,
+                             uint16_t* Xd_save, uint32_t* keep_save, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   DropoutSpec dr;
   if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  if (int rc = dropout_state(Xd_save, keep_save, &dr)) return rc;
   return fwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, Y, U_save, workspace, workspace_bytes, stream,
                   dr);
 }
@@ -1063,6 +1080,30 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   const int rpad = (r + 63) / 64 * 64;
   const int N = static_cast<int>(n_out), K = static_cast<int>(k_in);
 
+  // the adapter's input: X, or X * keep with dropout (the 1/(1-p) goes into the scales); the
+  // keep bits are read by the masked dX term.  Both come from the forward when it kept them.
+  const uint16_t* Xa = X;
+  const uint16_t* keep_bits = nullptr;
+  if (dr.on && dr.xd) {
+    Xa = dr.xd;
+    keep_bits = dr.bits;
+  } else if (dr.on) {
+    uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
+    uint16_t* bits = reinterpret_cast<uint16_t*>(ws + L.bits);
+    if (int rc = launch_dropout_mask(X, M, K, dr, Xm, sms, st, bits)) return rc;
+    Xa = Xm;
+    keep_bits = bits;
+  }
+  // U (from the forward, or recomputed)
+  const uint16_t* U = U_saved;
+  if (!U) {
+    // the forward's grid for U (split or not), so the recomputed U is bit-identical to a saved one
+    const int fmh = M > 256 ? 2 : 1;
+    const int fwd_pairs = static_cast<int>((M + 256 * fmh - 1) / (256 * fmh)) * ((N + 255) / 256);
+    const bool fwd_beside = M > 128 && adapter_beside(M, rpad, fwd_pairs, sms);
+    if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev, fwd_beside)) return rc;
+    U = Ubuf;
+  }
   // V = dY B  (B viewed MN-major: its rows are the reduction index)
   {
     CUtensorMap ta, tb;
@@ -1070,8 +1111,8 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     const int k_steps = N / 64;
     const int tiles = static_cast<int>((M + 127) / 128) * (rpad / 64);
     // The grid depends on the shapes alone, so V (and with it dA) is the same
-    // bit for bit whichever outputs are requested; it runs beside dX when V is
-    // dX's direct predecessor (U saved, no dropout kernel between).
+    // bit for bit whichever outputs are requested.  V is launched last before dX
+    // (after any mask pass and U recompute), so it can run beside dX.
     const int mh = M > 256 ? 2 : 1;
     const int pairs = static_cast<int>((M + 256 * mh - 1) / (256 * mh)) * ((K + 255) / 256);
     const bool beside = kVBesideDx && M > 128 && adapter_beside(M, rpad, pairs, sms);
@@ -1085,24 +1126,6 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
     if (int rc = launch_lora<false, true>(ta, tb, ta, tb, la, tiles, S, st, dev, QLORA_KERNEL_LORA_GEMM,
                                           beside ? 2 : 1))
       return rc;
-  }
-  // the adapter's input: X, or X * keep with dropout (the 1/(1-p) goes into the scales)
-  const uint16_t* Xa = X;
-  if (dr.on) {
-    uint16_t* Xm = reinterpret_cast<uint16_t*>(ws + L.xm);
-    uint16_t* keep_bits = reinterpret_cast<uint16_t*>(ws + L.bits);   // read by the masked dX term
-    if (int rc = launch_dropout_mask(X, M, K, dr, Xm, sms, st, keep_bits)) return rc;
-    Xa = Xm;
-  }
-  // U (from the forward, or recomputed)
-  const uint16_t* U = U_saved;
-  if (!U) {
-    // the forward's grid for U (split or not), so the recomputed U is bit-identical to a saved one
-    const int fmh = M > 256 ? 2 : 1;
-    const int fwd_pairs = static_cast<int>((M + 256 * fmh - 1) / (256 * fmh)) * ((N + 255) / 256);
-    const bool fwd_beside = M > 128 && adapter_beside(M, rpad, fwd_pairs, sms);
-    if (int rc = run_lora_down(Xa, M, K, A, r, dr.inv, s, Ubuf, nullptr, sms, st, dev, fwd_beside)) return rc;
-    U = Ubuf;
   }
   // The gradient kernel goes to the device's second stream, forked here and
   // launched after dX so that dX's CTAs are queued first; with per-kernel
@@ -1176,7 +1199,7 @@ static int bwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
       gd.out = dX;
       gd.ld_out = K;
       gd.drop_scale = s * dr.inv;
-      gd.drop_bits = reinterpret_cast<const uint32_t*>(ws + L.bits);
+      gd.drop_bits = reinterpret_cast<const uint32_t*>(keep_bits);
       // 128 x 128 tiles, one stage, four epilogue warps: two CTAs per SM, so one CTA's
       // loads overlap another's masked update
       const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 127) / 128), 1);
@@ -1238,10 +1261,11 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2, i
 int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t n_out, int64_t k_in,
                              const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float alpha,
                              float p, uint64_t seed, uint64_t offset, const uint16_t* dY, const uint16_t* U_saved,
-                             uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+                             const uint16_t* Xd_saved, const uint32_t* keep_saved, uint16_t* dX, float* dA, float* dB,
+                             void* workspace, size_t workspace_bytes, void* stream) {
   DropoutSpec dr;
   if (!make_dropout(p, seed, offset, &dr)) return QLORA_ERR_INVALID_ARG;
+  if (int rc = dropout_state(Xd_saved, keep_saved, &dr)) return rc;
   return bwd_impl(codes, q8, s2, n_out, k_in, X, M, A, B, r, alpha, dY, U_saved, dX, dA, dB, workspace,
                   workspace_bytes, stream, dr);
 }

@@ -283,11 +283,24 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
  * [0, 1) (else QLORA_ERR_INVALID_ARG); p == 0 is exactly the plain call.
  * Pass the same (p, seed, offset) to the forward and the backward of a step.
  * The workspace must hold qlora_workspace_bytes_dropout(M, N, K, r) bytes
- * (the plain size plus a bf16 M x K masked copy of X).  Arguments otherwise
- * as qlora_linear_fwd / qlora_linear_bwd.  Launches: mask, U, the fused
- * GEMM (forward); mask, V, [U], dY dequant(W), the masked adapter term of dX,
- * dA/dB (backward).  M <= 32 takes the tiled path (the few-token kernel
- * forms U from the unmasked tile).
+ * (the plain size plus a bf16 M x K masked copy of X and the keep bits).
+ *
+ * Kept dropout state (optional; both pointers or neither, 16-byte aligned):
+ *   Xd_save   bf16 [M x K]: the forward writes X * keep (dropped elements +0,
+ *             the 1/(1 - p) not applied), the adapter's input;
+ *   keep_save uint32 [M*K/32]: bit (e mod 32) of word e/32 is the keep
+ *             decision of element e = m*K + k.
+ * Given the same buffers as Xd_saved / keep_saved, the backward reads them
+ * instead of generating the mask again (what an autograd framework saves for
+ * dropout's backward), which takes one pass over X out of the backward; the
+ * results are bit-identical either way.  NULL, NULL: the backward generates
+ * the mask from (seed, offset) as the forward did.  Ignored when p == 0.
+ *
+ * Arguments otherwise as qlora_linear_fwd / qlora_linear_bwd.  Launches: mask,
+ * U, the fused GEMM (forward); [mask], [U], V, dY dequant(W), the masked
+ * adapter term of dX, dA/dB (backward; the mask pass only without kept state,
+ * U only when U_saved is NULL).  M <= 32 takes the tiled path (the few-token
+ * kernel forms U from the unmasked tile).
  */
 size_t qlora_workspace_bytes_dropout(int64_t M, int64_t n_out, int64_t k_in, int r);
 
@@ -297,6 +310,7 @@ int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* q8, const floa
                              const uint16_t* A, const uint16_t* B, int r, float alpha,
                              float p, uint64_t seed, uint64_t offset,
                              uint16_t* Y, uint16_t* U_save,
+                             uint16_t* Xd_save, uint32_t* keep_save,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* q8, const float* s2,
@@ -305,6 +319,7 @@ int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* q8, const floa
                              const uint16_t* A, const uint16_t* B, int r, float alpha,
                              float p, uint64_t seed, uint64_t offset,
                              const uint16_t* dY, const uint16_t* U_saved,
+                             const uint16_t* Xd_saved, const uint32_t* keep_saved,
                              uint16_t* dX, float* dA, float* dB,
                              void* workspace, size_t workspace_bytes, void* stream);
 

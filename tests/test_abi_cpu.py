@@ -142,10 +142,19 @@ def test_dropout_host_validation_without_gpu(lib):
     null = None
     for p in (-0.1, 1.0, 1.5, float("nan")):
         assert lib.qlora_linear_fwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
-                                            p, 1, 0, _p(P), null, _p(P), 1 << 30, null) == -1
+                                            p, 1, 0, _p(P), null, null, null, _p(P), 1 << 30, null) == -1
         assert lib.qlora_linear_bwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
-                                            p, 1, 0, _p(P), null, null, _p(P), _p(P), _p(P), 1 << 30,
+                                            p, 1, 0, _p(P), null, null, null, null, _p(P), _p(P), _p(P), 1 << 30,
                                             null) == -1
+    # kept dropout state: the masked input and the keep bits go together, 16-byte aligned
+    assert lib.qlora_linear_fwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                        0.1, 1, 0, _p(P), null, _p(P), null, _p(P), 1 << 30, null) == -1
+    assert lib.qlora_linear_bwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                        0.1, 1, 0, _p(P), null, null, _p(P), null, _p(P), _p(P), _p(P), 1 << 30,
+                                        null) == -1
+    assert lib.qlora_linear_fwd_dropout(_p(P), _p(P), _p(P), 256, 256, _p(P), 16, _p(P), _p(P), 8, 16.0,
+                                        0.1, 1, 0, _p(P), null, _p(P + 4), _p(P), _p(P), 1 << 30, null) == -2
+    for p in (-0.1, 1.0, 1.5, float("nan")):
         assert lib.qlora_dropout_apply(_p(P), 16, 256, p, 1, 0, _p(P), null) == -1
     assert lib.qlora_dropout_apply(_p(P), 16, 100, 0.1, 1, 0, _p(P), null) == -2   # K % 64
     assert lib.qlora_dropout_apply(_p(P), -1, 256, 0.1, 1, 0, _p(P), null) == -2

@@ -86,6 +86,34 @@ def test_dropout_adapter_dominant(M, N, K, r, p, w_kind):
     run_dropout_case(inp, p, seed=77 + M, offset=M * 31)
 
 
+@pytest.mark.parametrize("M,N,K,r,p", [(40, 512, 768, 16, 0.3), (300, 512, 768, 64, 0.05)])
+def test_kept_dropout_state(M, N, K, r, p):
+    """The forward's kept state: Xd_save is bit for bit the masked input and keep_save the
+    oracle's keep mask, packed one bit per element; a backward that reads them gives the bits
+    of one that generates the mask again."""
+    inp = synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=1700 + M)
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    X, A, B, dY = (to_dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
+    alpha, seed, offset = inp["alpha"], 99 + M, 5 * M
+    U = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    Xd = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda")
+    keep = torch.full((M * K // 32,), -1, dtype=torch.int32, device="cuda")
+    Y = q.qlora_linear_fwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, seed, offset, U_save=U, Xd_save=Xd,
+                                   keep_save=keep)
+    Y0 = q.qlora_linear_fwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, seed, offset)
+    assert torch.equal(Y, Y0)
+    assert torch.equal(Xd, q.qlora_dropout_apply(X, p, seed, offset))
+    bits = keep.cpu().numpy().view(np.uint32)
+    got = ((bits[:, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.uint8).reshape(M, K)
+    assert np.array_equal(got, oracle.dropout_keep(M, K, p, seed, offset))
+    g_kept = q.qlora_linear_bwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, seed, offset, dY, U_saved=U,
+                                        Xd_saved=Xd, keep_saved=keep)
+    g_gen = q.qlora_linear_bwd_dropout(codes, q8, s2, N, K, X, A, B, alpha, p, seed, offset, dY, U_saved=U)
+    assert q.qlora_device_status() == 0
+    for a, b in zip(g_kept, g_gen):
+        assert torch.equal(a, b)
+
+
 def test_dropout_train4096_sampled_rows():
     inp = synth.layer_inputs("train4096")
     rows = np.unique(np.concatenate([np.arange(0, 4096, 131), [0, 4095]]))
