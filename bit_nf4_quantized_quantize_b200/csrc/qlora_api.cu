@@ -25,6 +25,7 @@
 #include "lora_tc.cuh"
 #include "fused2_tc.cuh"
 #include "decode_tc.cuh"
+#include "decode_lut.cuh"
 #include "merge.cuh"
 #include "dropout.cuh"
 
@@ -375,6 +376,77 @@ int run_decode(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t
 }
 
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+constexpr int kLutRouteTokens = 4;   // the forward takes the table-lookup path up to this many tokens
+
+// One to eight tokens (decode_lut.cuh): U = X A^T in a small launch that also
+// prefetches the weight into L2, then the table-lookup kernel.  A CTA owns
+// T = ceil(N / 16 / SMs) tiles of 16 rows and all of K.  Returns
+// QLORA_ERR_UNSUPPORTED_SHAPE (nothing launched) when the shape is outside the
+// kernel's limits; the caller then takes the other few-token path.
+int run_decode_lut(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K,
+                   const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* Y,
+                   uint16_t* U_save, float* U32, int sms, cudaStream_t st, int dev) {
+  if (M > kLutMaxTokens || (q8 && !aligned16(q8)) || N * (K / 64) >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int tiles_total = static_cast<int>(N / kLutTile);
+  const int T = (tiles_total + sms - 1) / sms;
+  const int grid = (tiles_total + T - 1) / T;
+  const int mi = static_cast<int>(M), ki = static_cast<int>(K);
+  int n_slots = std::min(T, kLutMaxSlots);
+  while (n_slots > 1 && lut_layout(mi, ki, T, n_slots, r, q8 == nullptr).total > kLutMaxSmem) --n_slots;
+  const int smem = lut_layout(mi, ki, T, n_slots, r, q8 == nullptr).total;
+  if (smem > kLutMaxSmem) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  LutArgs a{};
+  a.codes = codes;
+  a.q8 = q8;
+  a.s2 = s2;
+  a.x = X;
+  a.b = B;
+  a.u = U32;
+  a.y = Y;
+  a.m = mi;
+  a.n = static_cast<int>(N);
+  a.k = ki;
+  a.r = r;
+  a.tiles_per_cta = T;
+  a.n_slots = n_slots;
+  a.s = s;
+  for (int i = 0; i < 16; ++i) a.level[i] = tables().level[i];
+  DecUArgs u{};
+  u.x = X;
+  u.a = A;
+  u.m = mi;
+  u.k = ki;
+  u.r = r;
+  u.u32 = U32;
+  u.u_save = U_save;
+  u.codes = codes;
+  u.consts = q8 ? q8 : reinterpret_cast<const uint8_t*>(s2);
+  u.consts_size = q8 ? 1 : 4;
+  u.n = static_cast<int>(N);
+  u.rows_per_cta = T * kLutTile;
+  static bool attr_set[kMaxDevices];
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(qlora_decode_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutMaxSmem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const unsigned u_grid = static_cast<unsigned>(std::max(grid, r));
+  if (int rc = timed(QLORA_KERNEL_LORA_GEMM, st, [&] {
+        if (M == 1) return launch_ex(qlora_decode_u_kernel<1>, dim3(u_grid), dim3(kDecUThreads), 0, st, 1, 1, u);
+        if (M == 2) return launch_ex(qlora_decode_u_kernel<2>, dim3(u_grid), dim3(kDecUThreads), 0, st, 1, 1, u);
+        if (M <= 4) return launch_ex(qlora_decode_u_kernel<4>, dim3(u_grid), dim3(kDecUThreads), 0, st, 1, 1, u);
+        return launch_ex(qlora_decode_u_kernel<8>, dim3(u_grid), dim3(kDecUThreads), 0, st, 1, 1, u);
+      }))
+    return rc;
+  return timed(QLORA_KERNEL_FWD_DECODE, st, [&] {
+    return launch_ex(qlora_decode_lut_kernel, dim3(static_cast<unsigned>(grid)), dim3(kLutThreads),
+                     static_cast<size_t>(smem), st, 1, 1, a);
+  });
+}
 
 struct WsLayout {
   size_t us, v, vs, u, xm, bits, total;
@@ -939,6 +1011,13 @@ static int fwd_impl(const uint8_t* codes, const uint8_t* q8, const float* s2, in
   const float s = alpha / static_cast<float>(r);
   const int rpad = (r + 63) / 64 * 64;
 
+  // one to four tokens: table-lookup kernel (two launches); measured faster than the
+  // tensor-memory kernel below up to four tokens (decode_lut.cuh)
+  if (M <= kLutRouteTokens && !dr.on) {
+    const int rc = run_decode_lut(codes, q8, s2, n_out, k_in, X, M, A, B, r, s, Y, U_save,
+                                  reinterpret_cast<float*>(ws + L.v), sms, st, dev);
+    if (rc != QLORA_ERR_UNSUPPORTED_SHAPE) return rc;
+  }
   // a few tokens: one launch, weight rows on the MMA's M side, U computed in-kernel
   if (M <= kDecMaxTokens && r <= kDecMaxRank && !dr.on)
     return run_decode(codes, q8, s2, n_out, k_in, X, M, A, B, r, s, Y, U_save, st, dev);

@@ -199,6 +199,14 @@ size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r);
  *   X  bf16[M*K], A bf16[r*K], B bf16[N*r]  read.
  *   Y  bf16[M*N]  written.
  *   U_save bf16[M*r] written with U (for the backward pass) unless NULL.
+ * Launches by batch size: M <= 4, two (U, which also prefetches the packed
+ * weight into L2, then a kernel that turns each code byte into a pair of fp16
+ * NF4 levels through a shared-memory table and applies c1 to each 64-column
+ * block's fp32 dot product, so it multiplies by the fp32 dequantized value
+ * level * c1 (to the level's fp16 rounding) rather than its bf16 rounding: a
+ * difference of about 2^-9 of each weight, well within the layer's tolerance);
+ * M <= 32, one (few-token
+ * tensor-memory kernel); larger M, U and then the fused GEMM.
  */
 int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      int64_t n_out, int64_t k_in,
@@ -368,7 +376,7 @@ int qlora_device_status(void* stream);
 #define QLORA_KERNEL_DX 5          /* fused transposed-dequant GEMM: dX       */
 #define QLORA_KERNEL_GRAD_GEMM 6   /* dA^T = X^T V, dB = dY^T U (partials)    */
 #define QLORA_KERNEL_GRAD_REDUCE 7 /* reduction of dA / dB partials          */
-#define QLORA_KERNEL_FWD_DECODE 8  /* small-M forward (M <= 32, r <= 64)     */
+#define QLORA_KERNEL_FWD_DECODE 8  /* small-M forward (M <= 32)              */
 #define QLORA_KERNEL_MERGE 9       /* adapter merge into the 16-bit base      */
 #define QLORA_KERNEL_DROPOUT 10    /* dropout mask / masked adapter dX        */
 #define QLORA_KERNEL_COUNT 11
