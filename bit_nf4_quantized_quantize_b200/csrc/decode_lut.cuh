@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   griddep_launch_dependents();   // the next grid may be scheduled now
   // the compute threads' global loads go out first: X pieces, B rows, group scales
   const int xpieces = m * K / 8;
-  constexpr int kXReg = 2;   // X pieces held in registers per thread (the rest are loaded later)
+  constexpr int kXReg = 4;   // X pieces loaded into registers up front per thread (M K <= 16384); the rest later
   uint4 xq[kXReg];
   uint4 bq = make_uint4(0u, 0u, 0u, 0u);
   float sgq = 0.f;
@@ -530,20 +530,22 @@ __global__ void __launch_bounds__(kDecUThreads) qlora_decode_u_kernel(const DecU
       const int c = c0 + i * kDecUThreads * 8;
       av[i] = c < k ? *reinterpret_cast<const uint4*>(arow + c) : make_uint4(0u, 0u, 0u, 0u);
     }
+    uint4 xv[MT][4];   // every token's loads of this pass go out together
 #pragma unroll
-    for (int tk = 0; tk < MT; ++tk) {
-      if (tk >= m) break;
-      uint4 xv[4];
+    for (int tk = 0; tk < MT; ++tk)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int c = c0 + i * kDecUThreads * 8;
-        xv[i] = c < k ? *reinterpret_cast<const uint4*>(args.x + static_cast<int64_t>(tk) * k + c)
-                      : make_uint4(0u, 0u, 0u, 0u);
+        xv[tk][i] = (tk < m && c < k) ? *reinterpret_cast<const uint4*>(args.x + static_cast<int64_t>(tk) * k + c)
+                                      : make_uint4(0u, 0u, 0u, 0u);
       }
+#pragma unroll
+    for (int tk = 0; tk < MT; ++tk) {
+      if (tk >= m) break;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t aw[4] = {av[i].x, av[i].y, av[i].z, av[i].w};
-        const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+        const uint32_t xw[4] = {xv[tk][i].x, xv[tk][i].y, xv[tk][i].z, xv[tk][i].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           acc[tk] = __fmaf_rn(__uint_as_float(aw[q] << 16), __uint_as_float(xw[q] << 16), acc[tk]);
