@@ -89,12 +89,20 @@ struct LutArgs {
 // pairs with their 8-byte loads); a multiple of 16 bytes.
 __host__ __device__ constexpr int lut_row_stride(int k) { return k / 2 + 4 * ((8 - (k / 8) % 32 + 32) % 32); }
 
+// Row stride of X in shared memory (halves): K padded by 8, so that the rows
+// of different tokens fall in different banks.
+__host__ __device__ constexpr int lut_x_stride(int k) { return k + 8; }
+// Floats per (row, token) of the partial totals: the 16 warps' values and one
+// of padding, so that consecutive rows fall in different banks.
+constexpr int kLutPartStride = kLutWarps + 1;
+
 // Shared-memory layout of one CTA; every part starts on a 16-byte boundary.
 //   table | ring (slots x 16 padded rows) | block constants of the CTA's rows (the
 //   16-byte aligned span holding them: q8 bytes, or fp32 absmax when single) |
-//   group scales s2 of those rows | c1 of every block of those rows (fp32) |
-//   X (fp16, scaled per 64-column block) | 2^e per token and block | partial
-//   totals [T][16][m][16 warps] | U (fp32) | B rows (bf16) | barriers: full, empty
+//   group scales s2 of those rows | c1 of every block of those rows (fp32,
+//   [block][row], rows padded by one) | X (fp16, scaled per 64-column block,
+//   rows of lut_x_stride) | 2^e per block and token | partial totals
+//   [T * 16 rows][m][kLutPartStride] | U (fp32) | B rows (bf16) | barriers: full, empty
 //   per slot, constants | abort word
 struct LutLayout {
   int ring, consts, s2g, c1, x, xsc, part, u, b, bars, abort_word, total;
@@ -108,10 +116,10 @@ __host__ __device__ inline LutLayout lut_layout(int m, int k, int tiles, int n_s
   L.consts = L.ring + n_slots * kLutTile * lut_row_stride(k);
   L.s2g = L.consts + lut_align16(rows * kblocks * (single ? 4 : 1) + 32);
   L.c1 = L.s2g + lut_align16((single ? 0 : rows * kblocks / 256 + 2) * 4);
-  L.x = L.c1 + lut_align16(rows * kblocks * 4);
-  L.xsc = L.x + lut_align16(m * k * 2);
+  L.x = L.c1 + lut_align16((rows + 1) * kblocks * 4);
+  L.xsc = L.x + lut_align16(m * lut_x_stride(k) * 2);
   L.part = L.xsc + lut_align16(m * kblocks * 4);
-  L.u = L.part + lut_align16(rows * m * kLutWarps * 4);
+  L.u = L.part + lut_align16(rows * m * kLutPartStride * 4);
   L.b = L.u + lut_align16(m * r * 4);
   L.bars = L.b + lut_align16(rows * r * 2);
   L.abort_word = L.bars + (2 * kLutMaxSlots + 1) * 8;
@@ -330,8 +338,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
                                                __fmul_rn(__uint_as_float(w[q] & 0xFFFF0000u), down));
           h[q] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        *reinterpret_cast<uint4*>(xs + i * 8) = make_uint4(h[0], h[1], h[2], h[3]);
-        if ((lane & 7) == 0) xsc[i / 8] = exp2_int(e);   // block i / 8 = token * kblocks + column block
+        const int tk = i / (K / 8), col8 = i - tk * (K / 8);   // token, 8-column piece
+        *reinterpret_cast<uint4*>(xs + tk * lut_x_stride(K) + col8 * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+        if ((lane & 7) == 0) xsc[(col8 / 8) * m + tk] = exp2_int(e);   // [block][token]
       }
     }
     if (ctid < rows_here * r / 8) *reinterpret_cast<uint4*>(bs + ctid * 8) = bq;
@@ -359,31 +368,35 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
     const bool tok_ok = g < m;                                   // this lane's B operand column is a real token
     // 32-bit shared-memory offsets of this lane's operands (block seg adds seg * 32, seg * 64 or seg)
     const uint32_t code_g = static_cast<uint32_t>(g * rs + 8 * t), code_h = code_g + 8u * static_cast<uint32_t>(rs);
-    const uint32_t x_off = static_cast<uint32_t>(g * K + 16 * t);          // in halves
-    const uint32_t xsc0 = static_cast<uint32_t>(2 * t * kblocks), xsc1 = xsc0 + static_cast<uint32_t>(kblocks);
+    const uint32_t x_off = static_cast<uint32_t>(g * lut_x_stride(K) + 16 * t);   // in halves
+    const uint32_t xsc0 = static_cast<uint32_t>(2 * t), xsc1 = xsc0 + 1u;         // + block * m
     const bool sx0_ok = 2 * t < m, sx1_ok = 2 * t + 1 < m;
     bool ok = rows_here == 0 || __all_sync(0xffffffffu, mbar_wait(consts_bar, 0, abort_flag));
     // c1 of every block of the CTA's rows, from the stored constants
     if (ok) {
       const uint32_t s2_first = static_cast<uint32_t>(row0) * static_cast<uint32_t>(kblocks);
       for (int i = ctid; i < rows_here * kblocks; i += kLutWarps * 32) {
+        const int rl = i / kblocks, bl = i - rl * kblocks;
+        float v;
         if (has_q8)
-          c1s[i] = lut_block_scale(true, consts[c_delta + i], s2g[((s2_first + i) >> 8) - static_cast<uint32_t>(g_lo)]);
+          v = lut_block_scale(true, consts[c_delta + i], s2g[((s2_first + i) >> 8) - static_cast<uint32_t>(g_lo)]);
         else
-          c1s[i] = *reinterpret_cast<const float*>(consts + c_delta + i * 4);
+          v = *reinterpret_cast<const float*>(consts + c_delta + i * 4);
+        c1s[bl * (rows_here + 1) + rl] = v;
       }
     }
     named_bar_sync(1, kLutWarps * 32);   // c1
     // one 64-column block: code bytes of rows g, g + 8 at code_g / code_h + blk * 32 of the slot
     const uint32_t lut_base = smem_u32(lut_smem);
     const uint32_t c1_base = smem_u32(c1s), xsc_base = smem_u32(xsc), x_base = smem_u32(xs) + 2u * x_off;
+    const uint32_t m_u = static_cast<uint32_t>(m);
     auto block = [&](uint32_t slot_base, uint32_t blk, uint32_t c1_row, float (&acc)[4]) {
       const uint2 wg = lds_v2(slot_base + code_g + blk * 32u);
       const uint2 wh = lds_v2(slot_base + code_h + blk * 32u);
-      const float cg = lds_f32(c1_base + 4u * (c1_row + blk));
-      const float ch = lds_f32(c1_base + 4u * (c1_row + 8u * kblocks + blk));
-      const float sx0 = sx0_ok ? lds_f32(xsc_base + 4u * (xsc0 + blk)) : 0.f;   // tokens past m: 0
-      const float sx1 = sx1_ok ? lds_f32(xsc_base + 4u * (xsc1 + blk)) : 0.f;
+      const float cg = lds_f32(c1_base + 4u * (blk * static_cast<uint32_t>(rows_here + 1) + c1_row));
+      const float ch = lds_f32(c1_base + 4u * (blk * static_cast<uint32_t>(rows_here + 1) + c1_row + 8u));
+      const float sx0 = sx0_ok ? lds_f32(xsc_base + 4u * (blk * m_u + xsc0)) : 0.f;   // tokens past m: 0
+      const float sx1 = sx1_ok ? lds_f32(xsc_base + 4u * (blk * m_u + xsc1)) : 0.f;
       uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = make_uint4(0u, 0u, 0u, 0u);
       if (tok_ok) {
         xa = lds_v4(x_base + blk * 128u);
@@ -414,7 +427,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
       ok = __all_sync(0xffffffffu, mbar_wait(full + slot, (c / n_slots) & 1, abort_flag));
       if (!ok) break;
       const uint32_t sbase = smem_u32(ring) + static_cast<uint32_t>(slot * slot_bytes);
-      const uint32_t c1_row = static_cast<uint32_t>((c * kLutTile + g) * kblocks);   // row g of the tile in c1s
+      const uint32_t c1_row = static_cast<uint32_t>(c * kLutTile + g);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};   // rows g, g + 8 x tokens 2t, 2t + 1
       int blk = seg_lo;
       for (; blk + 4 <= seg_hi; blk += 4) {   // four blocks at a time: offsets are immediates
@@ -423,14 +436,14 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
       }
       for (; blk < seg_hi; ++blk) block(sbase, static_cast<uint32_t>(blk), c1_row, acc);
       // partial totals of this warp, [tile row][token][warp]; then the slot is free
-      float* pt = part + static_cast<int64_t>(c * kLutTile) * m * kLutWarps;
+      float* pt = part + static_cast<int64_t>(c * kLutTile) * m * kLutPartStride;
       if (2 * t < m) {
-        pt[(g * m + 2 * t) * kLutWarps + warp] = acc[0];
-        pt[((g + 8) * m + 2 * t) * kLutWarps + warp] = acc[2];
+        pt[(g * m + 2 * t) * kLutPartStride + warp] = acc[0];
+        pt[((g + 8) * m + 2 * t) * kLutPartStride + warp] = acc[2];
       }
       if (2 * t + 1 < m) {
-        pt[(g * m + 2 * t + 1) * kLutWarps + warp] = acc[1];
-        pt[((g + 8) * m + 2 * t + 1) * kLutWarps + warp] = acc[3];
+        pt[(g * m + 2 * t + 1) * kLutPartStride + warp] = acc[1];
+        pt[((g + 8) * m + 2 * t + 1) * kLutPartStride + warp] = acc[3];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + slot);
@@ -456,7 +469,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   for (int idx = tid; idx < rows_here * m; idx += kLutThreads) {
     const int tk = idx / rows_here;
     const int rl = idx - tk * rows_here;
-    const float* pp = part + (static_cast<int64_t>(rl) * m + tk) * kLutWarps;
+    const float* pp = part + (static_cast<int64_t>(rl) * m + tk) * kLutPartStride;
     float y = 0.f;
 #pragma unroll
     for (int w = 0; w < kLutWarps; ++w) y = __fadd_rn(y, pp[w]);
