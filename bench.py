@@ -677,7 +677,8 @@ def run_ours(args, rank, world, local_rank):
         # profiling case for ncu: one step to load the modules, one step to
         # capture, then decode forwards (r = 8) on the same weight: two at
         # M = 1, then two at M = 16.  Launches: [L2 flush write + L2 flush read
-        # + 6 step kernels] x 2, then 4 decode kernels.
+        # + 6 step kernels] x 2, then [adapter kernel + table kernel] x 2 (M = 1)
+        # and 2 tensor-memory decode kernels (M = 16).
         from bit_nf4_quantized_quantize_b200 import synth
         dinp = synth.layer_inputs("decode", M=16)
         decA, decB = (torch.from_numpy(dinp[k].view(np.int16)).view(torch.bfloat16).to(dev) for k in ("A", "B"))

@@ -153,10 +153,10 @@ def test_zero_adapter_reduces_to_dequant_matmul():
 
 
 @pytest.mark.parametrize("M,N,K,r,w_kind", [
-    (1, 1024, 4096, 8, "zero"),       # few-token path, K split over a cluster
-    (4, 4096, 4096, 8, "zero"),       # the decode workload's shape
-    (16, 640, 1024, 64, "zero"),      # few-token path, rank 64
-    (16, 1024, 2048, 8, "normal"),    # few-token path, adapter well above the main term
+    (1, 1024, 4096, 8, "zero"),       # table-lookup path
+    (4, 4096, 4096, 8, "zero"),       # the decode workload's shape, table-lookup path
+    (16, 640, 1024, 64, "zero"),      # tensor-memory few-token path, rank 64
+    (16, 1024, 2048, 8, "normal"),    # tensor-memory few-token path, adapter well above the main term
     (40, 512, 768, 16, "zero"),       # tiled path, split K
     (100, 768, 1536, 64, "normal"),   # tiled path
     (300, 512, 768, 64, "zero"),      # CTA-pair path
@@ -184,8 +184,8 @@ def test_adapter_slices_filling_every_stage_back_to_back(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K,r", [
-    (1, 4096, 4096, 8),      # one token, K split over a cluster
-    (2, 320, 64, 8),         # one k-step (no split), ragged last row tile (320 = 2*128 + 64)
+    (1, 4096, 4096, 8),      # one token (table-lookup kernel)
+    (2, 320, 64, 8),         # two tokens, one 64-column block (table-lookup kernel)
     (5, 640, 1024, 24),      # rank not a multiple of 16
     (16, 1024, 640, 64),     # 16 tokens (one 16-token tile), rank 64
     (17, 384, 2048, 16),     # one past a 16-token tile
@@ -194,10 +194,11 @@ def test_adapter_slices_filling_every_stage_back_to_back(M, N, K):
     (64, 768, 1536, 64),     # the largest small-M case
 ])
 def test_small_m_forward_and_saved_u(M, N, K, r):
-    """Few-token forward (M <= 32): weight rows and adapter rows share the
-    MMA's row side, the K range is split over a cluster, U = X A^T is formed
-    per K range in the same launch.  M = 33 and 64 cross into the tiled path.
-    Y and the saved U against the oracle; the backward then uses that saved U."""
+    """Few-token forward: M <= 4 take the table-lookup kernel (tests/test_decode_lut_gpu.py
+    has its own cases); 5 <= M <= 32 the tensor-memory kernel, where weight rows and
+    adapter rows share the MMA's row side, the K range is split over a cluster and
+    U = X A^T is formed per K range in the same launch.  M = 33 and 64 cross into the
+    tiled path.  Y and the saved U against the oracle; the backward then uses that saved U."""
     run_case(synth.layer_inputs("tiny", M=M, shape=(N, K), r=r, seed=500 + M))
 
 

@@ -40,7 +40,8 @@ def _noalloc_call(lib, codes, q8, s2, N, K, X, A, B, alpha, Y, U, M=None):
                                         _p(A), _p(B), A.shape[0], float(alpha), _p(Y), _p(U), stream)
 
 
-CASES = [dict(M=4, shape=(1024, 2048), r=8, seed=40),     # few-token path, K split over a cluster
+CASES = [dict(M=4, shape=(1024, 2048), r=8, seed=40),     # few-token table-lookup path
+         dict(M=16, shape=(1024, 2048), r=8, seed=44),    # few-token tensor-memory path, K split over a cluster
          dict(M=100, shape=(768, 1536), r=64, seed=43),    # single-CTA tiled path
          dict(M=300, shape=(512, 768), r=16, seed=41),     # CTA-pair path
          dict(M=1024, shape=(1024, 512), r=64, seed=42)]   # CTA-pair path, several waves
