@@ -131,6 +131,18 @@ __device__ __forceinline__ void add2_rn(float& d0, float& d1, float a0, float a1
       : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b));
 }
 
+// Three-input fp32 max and min (exact, like a chain of two fmaxf / fminf).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)) : "memory");
@@ -149,21 +161,27 @@ __device__ __forceinline__ uint32_t nf4_code8(const float (&f)[8], float am, boo
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rcp) : "f"(am));   // am and 1/am are normal here
     const float r16 = 16.f * rcp;   // exact scaling
     float dmin = 1.f;
-    packed = 0;
+    uint32_t pair[4];   // byte j / 2: the codes of f[j] (low nibble) and f[j + 1]
 #pragma unroll
-    for (int j = 6; j >= 0; j -= 2) {
+    for (int j = 0; j < 8; j += 2) {
       float t[2], u[2];
+      uint32_t x[2];
       fma2_rn(t[0], t[1], f[j], f[j + 1], r16, kCellOffset);
       add2_rn(u[0], u[1], t[0], t[1], kQuarterMagic);
+      float d[2];
 #pragma unroll
-      for (int h = 1; h >= 0; --h) {
+      for (int h = 0; h < 2; ++h) {
         const uint32_t off = __float_as_uint(u[h]) & 0xFCu;
         const uint32_t ent = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(sm.fast) + off);
-        const float d = __uint_as_float(ent) - t[h];
-        dmin = fminf(dmin, fabsf(d));
-        packed = (packed << 4) + (ent & 15u) + (__float_as_uint(d) >> 31);
+        d[h] = __uint_as_float(ent) - t[h];
+        // the code in the low 4 bits: the cell's left-edge code, plus one above its midpoint
+        // (a cell whose left-edge code is 15 holds no midpoint, so the nibble never carries)
+        x[h] = ent + (__float_as_uint(d[h]) >> 31);
       }
+      dmin = min3f(dmin, fabsf(d[0]), fabsf(d[1]));
+      pair[j / 2] = (x[1] << 4) + (x[0] & 15u);   // bits above 7 are dropped by the byte permutes
     }
+    packed = __byte_perm(__byte_perm(pair[0], pair[1], 0x0040u), __byte_perm(pair[2], pair[3], 0x0040u), 0x5410u);
     need = dmin <= kFastGuard;
   }
   if (__any_sync(0xffffffffu, need)) {
@@ -290,9 +308,8 @@ quantize_nf4_kernel(const float* __restrict__ W, int64_t n_blocks, int64_t group
       const float4 a = *reinterpret_cast<const float4*>(src + 4 * swz);
       const float4 b = *reinterpret_cast<const float4*>(src + 4 * (swz ^ 1));
       const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      float am = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
+      float am = max3f(max3f(fabsf(f[0]), fabsf(f[1]), fabsf(f[2])), max3f(fabsf(f[3]), fabsf(f[4]), fabsf(f[5])),
+                       fmaxf(fabsf(f[6]), fabsf(f[7])));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
