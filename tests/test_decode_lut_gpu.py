@@ -102,3 +102,21 @@ def test_deterministic_and_two_launches():
             outs.append((Y, U))
         assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
     assert q.qlora_device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K,launches", [
+    (1, 4096, 11008, 2),     # the 7B down projection: one 88 KB ring slot, the CTA's tiles through it in turn
+    (2, 11008, 4096, 2),     # the 7B gate / up projection: five tiles per CTA
+    (3, 4096, 11008, 1),     # three tokens of the down projection exceed the shared memory: tensor-memory path
+])
+def test_llama7b_shapes(M, N, K, launches):
+    """The 7B stack's wide shapes at a few tokens: the table path where its shared memory
+    fits, the tensor-memory path where it does not; the same bounds either way."""
+    inp = synth.layer_inputs("tiny", M=M, shape=(N, K), r=8, seed=1900 + M)
+    codes, q8, s2 = q.qlora_quantize_nf4_dq(torch.from_numpy(inp["W"]).cuda())
+    X, A, B = (to_dev_bf16(inp[k]) for k in ("X", "A", "B"))
+    n0 = q.qlora_launch_count()
+    q.qlora_linear_fwd(codes, q8, s2, N, K, X, A, B, inp["alpha"])
+    torch.cuda.synchronize()
+    assert q.qlora_launch_count() - n0 == launches
+    run_case(inp, check_bwd=False)
