@@ -103,7 +103,7 @@ constexpr int kLutPartStride = kLutWarps + 1;
 //   [block][row], rows padded by one) | X (fp16, scaled per 64-column block,
 //   rows of lut_x_stride) | 2^e per block and token | partial totals
 //   [T * 16 rows][m][kLutPartStride] | U (fp32) | B rows (bf16) | barriers: full, empty
-//   per slot, constants | abort word
+//   per slot, constants, X | abort word
 struct LutLayout {
   int ring, consts, s2g, c1, x, xsc, part, u, b, bars, abort_word, total;
 };
@@ -122,7 +122,7 @@ __host__ __device__ inline LutLayout lut_layout(int m, int k, int tiles, int n_s
   L.u = L.part + lut_align16(rows * m * kLutPartStride * 4);
   L.b = L.u + lut_align16(m * r * 4);
   L.bars = L.b + lut_align16(rows * r * 2);
-  L.abort_word = L.bars + (2 * kLutMaxSlots + 1) * 8;
+  L.abort_word = L.bars + (2 * kLutMaxSlots + 2) * 8;
   L.total = L.abort_word + 16;
   return L;
 }
@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(lut_smem + L.bars);   // [slot]
   uint64_t* empty = full + kLutMaxSlots;                              // [slot]
   uint64_t* consts_bar = empty + kLutMaxSlots;
+  uint64_t* x_bar = consts_bar + 1;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(lut_smem + L.abort_word);
   int* issued = reinterpret_cast<int*>(lut_smem + L.abort_word) + 1;   // tiles the producer copied
 
@@ -255,18 +256,11 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   const int64_t g_lo = (static_cast<int64_t>(row0) * kblocks) >> 8;   // first group scale of the CTA's rows
 
   griddep_launch_dependents();   // the next grid may be scheduled now
-  // the compute threads' global loads go out first: X pieces, B rows, group scales
+  // the compute threads' global loads go out first: B rows, group scales (X comes by bulk copy)
   const int xpieces = m * K / 8;
-  constexpr int kXReg = 4;   // X pieces loaded into registers up front per thread (M K <= 16384); the rest later
-  uint4 xq[kXReg];
   uint4 bq = make_uint4(0u, 0u, 0u, 0u);
   float sgq = 0.f;
   if (warp < kLutWarps) {
-#pragma unroll
-    for (int j = 0; j < kXReg; ++j) {
-      const int i = tid + j * kLutWarps * 32;
-      xq[j] = i < xpieces ? ld_cg_v4(args.x + static_cast<int64_t>(i) * 8) : make_uint4(0u, 0u, 0u, 0u);
-    }
     if (tid < rows_here * r / 8) bq = ld_cg_v4(args.b + static_cast<int64_t>(row0) * r + tid * 8);
     if (has_q8 && rows_here > 0) {
       const int64_t g_hi = (static_cast<int64_t>(row0 + rows_here) * kblocks - 1) >> 8;
@@ -279,6 +273,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
       mbar_init(empty + i, kLutWarps);
     }
     mbar_init(consts_bar, 1);
+    mbar_init(x_bar, 1);
     *abort_flag = 0;
     *issued = 0;
     fence_barrier_init();
@@ -287,6 +282,13 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
 
   if (warp == kLutWarps) {
     // ---------------------------------------------------------------- producer
+    // X rows first (one bulk copy per token, bf16, into the token's padded row: converted in
+    // place), then the block constants
+    if (lane == 0) mbar_arrive_expect_tx(x_bar, static_cast<uint32_t>(m * K * 2));
+    __syncwarp();
+    if (lane < m)
+      lut_bulk_copy(xs + lane * lut_x_stride(K), args.x + static_cast<int64_t>(lane) * K, static_cast<uint32_t>(K * 2),
+                    x_bar);
     if (lane == 0 && rows_here > 0) {
       mbar_arrive_expect_tx(consts_bar, cbytes);
       lut_bulk_copy(consts, cspan, cbytes, consts_bar);
@@ -309,17 +311,29 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   } else {
     // ---------------------------------------------------------------- compute warps
     const int ctid = tid;   // 0 .. 511
-    // X: 16-byte pieces (8 values); the 8 pieces of a 64-column block sit in 8 consecutive lanes
-    for (int i0 = warp * 32, j = 0; i0 < xpieces; i0 += kLutWarps * 32, ++j) {
+    // table: entry for byte value e, lane copy c = fp16 (level[e & 15], level[e >> 4]) at e * 256 + c * 4
+    // (built while the X rows are in flight)
+    for (int i = ctid; i < 256 * 8; i += kLutWarps * 32) {
+      const int e = i >> 3;
+      const __half2 h = __floats2half2_rn(args.level[e & 15], args.level[e >> 4]);
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(&h);
+      *reinterpret_cast<uint4*>(lut_smem + e * 256 + (i & 7) * 16) = make_uint4(v, v, v, v);
+    }
+    if (ctid < rows_here * r / 8) *reinterpret_cast<uint4*>(bs + ctid * 8) = bq;
+    for (int i = ctid + kLutWarps * 32; i < rows_here * r / 8; i += kLutWarps * 32)
+      *reinterpret_cast<uint4*>(bs + i * 8) = ld_cg_v4(args.b + static_cast<int64_t>(row0) * r + i * 8);
+    if (has_q8 && rows_here > 0) {
+      const int64_t g_hi = (static_cast<int64_t>(row0 + rows_here) * kblocks - 1) >> 8;
+      if (ctid <= g_hi - g_lo) s2g[ctid] = sgq;
+      for (int i = ctid + kLutWarps * 32; i <= g_hi - g_lo; i += kLutWarps * 32) s2g[i] = __ldg(args.s2 + g_lo + i);
+    }
+    // X, in place: 16-byte pieces (8 values); the 8 pieces of a 64-column block sit in 8 consecutive lanes
+    const bool x_ok = __all_sync(0xffffffffu, mbar_wait(x_bar, 0, abort_flag));
+    for (int i0 = warp * 32; x_ok && i0 < xpieces; i0 += kLutWarps * 32) {
       const int i = i0 + lane;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (j < kXReg) {
-#pragma unroll
-        for (int q = 0; q < kXReg; ++q)
-          if (q == j) v = xq[q];
-      } else if (i < xpieces) {
-        v = ld_cg_v4(args.x + static_cast<int64_t>(i) * 8);
-      }
+      const int tk = i / (K / 8), col8 = i - tk * (K / 8);   // token, 8-column piece
+      uint4* px = reinterpret_cast<uint4*>(xs + tk * lut_x_stride(K) + col8 * 8);
+      const uint4 v = i < xpieces ? *px : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
       uint32_t mx = 0u;
 #pragma unroll
@@ -338,25 +352,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
                                                __fmul_rn(__uint_as_float(w[q] & 0xFFFF0000u), down));
           h[q] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        const int tk = i / (K / 8), col8 = i - tk * (K / 8);   // token, 8-column piece
-        *reinterpret_cast<uint4*>(xs + tk * lut_x_stride(K) + col8 * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+        *px = make_uint4(h[0], h[1], h[2], h[3]);
         if ((lane & 7) == 0) xsc[(col8 / 8) * m + tk] = exp2_int(e);   // [block][token]
       }
-    }
-    if (ctid < rows_here * r / 8) *reinterpret_cast<uint4*>(bs + ctid * 8) = bq;
-    for (int i = ctid + kLutWarps * 32; i < rows_here * r / 8; i += kLutWarps * 32)
-      *reinterpret_cast<uint4*>(bs + i * 8) = ld_cg_v4(args.b + static_cast<int64_t>(row0) * r + i * 8);
-    if (has_q8 && rows_here > 0) {
-      const int64_t g_hi = (static_cast<int64_t>(row0 + rows_here) * kblocks - 1) >> 8;
-      if (ctid <= g_hi - g_lo) s2g[ctid] = sgq;
-      for (int i = ctid + kLutWarps * 32; i <= g_hi - g_lo; i += kLutWarps * 32) s2g[i] = __ldg(args.s2 + g_lo + i);
-    }
-    // table: entry for byte value e, lane copy c = fp16 (level[e & 15], level[e >> 4]) at e * 256 + c * 4
-    for (int i = ctid; i < 256 * 8; i += kLutWarps * 32) {
-      const int e = i >> 3;
-      const __half2 h = __floats2half2_rn(args.level[e & 15], args.level[e >> 4]);
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(&h);
-      *reinterpret_cast<uint4*>(lut_smem + e * 256 + (i & 7) * 16) = make_uint4(v, v, v, v);
     }
     named_bar_sync(1, kLutWarps * 32);   // table, X, block scales of X, B rows
 
@@ -371,7 +369,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
     const uint32_t x_off = static_cast<uint32_t>(g * lut_x_stride(K) + 16 * t);   // in halves
     const uint32_t xsc0 = static_cast<uint32_t>(2 * t), xsc1 = xsc0 + 1u;         // + block * m
     const bool sx0_ok = 2 * t < m, sx1_ok = 2 * t + 1 < m;
-    bool ok = rows_here == 0 || __all_sync(0xffffffffu, mbar_wait(consts_bar, 0, abort_flag));
+    bool ok = x_ok && (rows_here == 0 || __all_sync(0xffffffffu, mbar_wait(consts_bar, 0, abort_flag)));
     // c1 of every block of the CTA's rows, from the stored constants
     if (ok) {
       const uint32_t s2_first = static_cast<uint32_t>(row0) * static_cast<uint32_t>(kblocks);
@@ -460,6 +458,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
         lut_drain(full + sl, (last / n_slots) & 1);
       }
       if (rows_here > 0) lut_drain(consts_bar, 0);
+      lut_drain(x_bar, 0);
     }
     return;
   }

@@ -387,7 +387,9 @@ constexpr int kLutRouteTokens = 4;   // the forward takes the table-lookup path 
 int run_decode_lut(const uint8_t* codes, const uint8_t* q8, const float* s2, int64_t N, int64_t K,
                    const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* Y,
                    uint16_t* U_save, float* U32, int sms, cudaStream_t st, int dev) {
-  if (M > kLutMaxTokens || (q8 && !aligned16(q8)) || N * (K / 64) >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  // the X rows and the 8-bit constants arrive by bulk copies: 16-byte aligned
+  if (M > kLutMaxTokens || !aligned16(X) || (q8 && !aligned16(q8)) || N * (K / 64) >= (int64_t(1) << 31))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int tiles_total = static_cast<int>(N / kLutTile);
   const int T = (tiles_total + sms - 1) / sms;
   const int grid = (tiles_total + T - 1) / T;
