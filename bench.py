@@ -279,6 +279,8 @@ DECODE_N = DECODE_K = 4096
 DECODE_RANK = 8
 DECODE_COPIES = 32          # rotated weight copies: 32 x 8.65 MB = 277 MB, more than L2
 DECODE_REPLAYS = 20
+DECODE_SINGLES = 12          # single launches timed one at a time
+DECODE_SLEEP_CYCLES = 200000  # about 100 us of GPU sleep before each single launch's first event
 
 
 def decode_weight_bytes(N, K):
@@ -291,7 +293,8 @@ def decode_weight_bytes(N, K):
 def run_decode(q, dev, peaks):
     """Forward of one 4096 x 4096 NF4+DQ layer (r = 8) at M in {1, 4, 16}: a
     CUDA graph of 32 layers, each on its own copy of the weight, replayed;
-    time per layer from CUDA events around the replays."""
+    time per layer from CUDA events around the replays.  Also the time of a
+    single stream launch between its own event pair."""
     import torch
     from bit_nf4_quantized_quantize_b200 import synth
     N, K, r = DECODE_N, DECODE_K, DECODE_RANK
@@ -332,13 +335,31 @@ def run_decode(q, dev, peaks):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / (DECODE_REPLAYS * DECODE_COPIES)
         gbs = wbytes / (us * 1e-6) / 1e9
-        out[str(M)] = {"us_per_layer": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+        # one launch alone (stream launch, no graph), each on a weight copy last read 31
+        # launches earlier (so out of L2), between its own event pair; a GPU-side sleep in
+        # front of the first event lets the host enqueue the launch before the GPU reaches it,
+        # so the time is the GPU's and not the host's launch overhead
+        single = []
+        for i in range(DECODE_SINGLES):
+            c = copies[i % DECODE_COPIES]
+            torch.cuda._sleep(DECODE_SLEEP_CYCLES)
+            e0.record()
+            q.qlora_linear_fwd(*c, N, K, X, A, B, inp["alpha"], Y=Y, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            single.append(e0.elapsed_time(e1) * 1e3)
+        single_us = float(np.median(single[2:]))
+        out[str(M)] = {"us_per_layer": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+                       "single_launch_us": single_us}
         del g
     rc = q.qlora_device_status()
     if rc != 0:
         raise RuntimeError(f"device status after the decode region: {q.qlora_strerror(rc)}")
     return {"workload": f"one {N}x{K} NF4+DQ layer, forward, r={r}, alpha=16; CUDA graph of {DECODE_COPIES} layers "
                         f"on rotated weight copies ({DECODE_COPIES * wbytes / 1e6:.0f} MB, more than L2)",
+            "single_launch_timing": "median of single stream launches between their own event pair, each on a weight "
+                                    "copy out of L2, enqueued behind a GPU sleep so that the host's launch time is "
+                                    "hidden; the launch latency after a timing event is included",
             "bound": "hbm", "algorithmic_bytes_per_layer": wbytes, "peak_gbs": peaks["hbm_gbs"],
             "unit": "GB/s", "by_tokens": out}
 
