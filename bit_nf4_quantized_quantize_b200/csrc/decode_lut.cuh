@@ -92,6 +92,11 @@ __host__ __device__ constexpr int lut_row_stride(int k) { return k / 2 + 4 * ((8
 // Row stride of X in shared memory (halves): K padded by 8, so that the rows
 // of different tokens fall in different banks.
 __host__ __device__ constexpr int lut_x_stride(int k) { return k + 8; }
+// Row stride (floats) of the c1 table ([row][block]) and of the activation scales
+// ([token][block]): at least the number of blocks, a multiple of 4 and 4 mod 32, so that a
+// lane's 16-byte load of four consecutive blocks is aligned and the 8 rows (tokens) a warp
+// reads at once fall in 8 distinct groups of 4 banks.
+__host__ __device__ constexpr int lut_scale_stride(int kblocks) { return kblocks + ((4 - kblocks) % 32 + 32) % 32; }
 // Floats per (row, token) of the partial totals: the 16 warps' values and one
 // of padding, so that consecutive rows fall in different banks.
 constexpr int kLutPartStride = kLutWarps + 1;
@@ -100,8 +105,8 @@ constexpr int kLutPartStride = kLutWarps + 1;
 //   table | ring (slots x 16 padded rows) | block constants of the CTA's rows (the
 //   16-byte aligned span holding them: q8 bytes, or fp32 absmax when single) |
 //   group scales s2 of those rows | c1 of every block of those rows (fp32,
-//   [block][row], rows padded by one) | X (fp16, scaled per 64-column block,
-//   rows of lut_x_stride) | 2^e per block and token | partial totals
+//   [row][block], rows of lut_scale_stride) | X (fp16, scaled per 64-column block,
+//   rows of lut_x_stride) | 2^e per token and block (rows of lut_scale_stride) | partial totals
 //   [T * 16 rows][m][kLutPartStride] | U (fp32) | B rows (bf16) | barriers: full, empty
 //   per slot, constants, X | abort word
 struct LutLayout {
@@ -116,9 +121,9 @@ __host__ __device__ inline LutLayout lut_layout(int m, int k, int tiles, int n_s
   L.consts = L.ring + n_slots * kLutTile * lut_row_stride(k);
   L.s2g = L.consts + lut_align16(rows * kblocks * (single ? 4 : 1) + 32);
   L.c1 = L.s2g + lut_align16((single ? 0 : rows * kblocks / 256 + 2) * 4);
-  L.x = L.c1 + lut_align16((rows + 1) * kblocks * 4);
+  L.x = L.c1 + lut_align16(rows * lut_scale_stride(kblocks) * 4);
   L.xsc = L.x + lut_align16(m * lut_x_stride(k) * 2);
-  L.part = L.xsc + lut_align16(m * kblocks * 4);
+  L.part = L.xsc + lut_align16(m * lut_scale_stride(kblocks) * 4);
   L.u = L.part + lut_align16(rows * m * kLutPartStride * 4);
   L.b = L.u + lut_align16(m * r * 4);
   L.bars = L.b + lut_align16(rows * r * 2);
@@ -244,6 +249,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
   const int rs = lut_row_stride(K);
   const int slot_bytes = kLutTile * rs;
   const int kblocks = K / 64;
+  const int ss = lut_scale_stride(kblocks);   // row stride of the c1 and X-scale tables
   const uint8_t* cta_codes = args.codes + static_cast<int64_t>(row0) * row_bytes;
   // the 16-byte aligned span holding the block constants of the CTA's rows
   const int csize = has_q8 ? 1 : 4;
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
           h[q] = *reinterpret_cast<const uint32_t*>(&hv);
         }
         *px = make_uint4(h[0], h[1], h[2], h[3]);
-        if ((lane & 7) == 0) xsc[(col8 / 8) * m + tk] = exp2_int(e);   // [block][token]
+        if ((lane & 7) == 0) xsc[tk * ss + col8 / 8] = exp2_int(e);   // [token][block]
       }
     }
     named_bar_sync(1, kLutWarps * 32);   // table, X, block scales of X, B rows
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
     // 32-bit shared-memory offsets of this lane's operands (block seg adds seg * 32, seg * 64 or seg)
     const uint32_t code_g = static_cast<uint32_t>(g * rs + 8 * t), code_h = code_g + 8u * static_cast<uint32_t>(rs);
     const uint32_t x_off = static_cast<uint32_t>(g * lut_x_stride(K) + 16 * t);   // in halves
-    const uint32_t xsc0 = static_cast<uint32_t>(2 * t), xsc1 = xsc0 + 1u;         // + block * m
+    const uint32_t xsc0 = static_cast<uint32_t>(2 * t * ss), xsc1 = xsc0 + static_cast<uint32_t>(ss);   // + block
     const bool sx0_ok = 2 * t < m, sx1_ok = 2 * t + 1 < m;
     bool ok = x_ok && (rows_here == 0 || __all_sync(0xffffffffu, mbar_wait(consts_bar, 0, abort_flag)));
     // c1 of every block of the CTA's rows, from the stored constants
@@ -380,21 +386,16 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
           v = lut_block_scale(true, consts[c_delta + i], s2g[((s2_first + i) >> 8) - static_cast<uint32_t>(g_lo)]);
         else
           v = *reinterpret_cast<const float*>(consts + c_delta + i * 4);
-        c1s[bl * (rows_here + 1) + rl] = v;
+        c1s[rl * ss + bl] = v;
       }
     }
     named_bar_sync(1, kLutWarps * 32);   // c1
     // one 64-column block: code bytes of rows g, g + 8 at code_g / code_h + blk * 32 of the slot
     const uint32_t lut_base = smem_u32(lut_smem);
     const uint32_t c1_base = smem_u32(c1s), xsc_base = smem_u32(xsc), x_base = smem_u32(xs) + 2u * x_off;
-    const uint32_t m_u = static_cast<uint32_t>(m);
-    auto block = [&](uint32_t slot_base, uint32_t blk, uint32_t c1_row, float (&acc)[4]) {
+    auto block = [&](uint32_t slot_base, uint32_t blk, float cg, float ch, float sx0, float sx1, float (&acc)[4]) {
       const uint2 wg = lds_v2(slot_base + code_g + blk * 32u);
       const uint2 wh = lds_v2(slot_base + code_h + blk * 32u);
-      const float cg = lds_f32(c1_base + 4u * (blk * static_cast<uint32_t>(rows_here + 1) + c1_row));
-      const float ch = lds_f32(c1_base + 4u * (blk * static_cast<uint32_t>(rows_here + 1) + c1_row + 8u));
-      const float sx0 = sx0_ok ? lds_f32(xsc_base + 4u * (blk * m_u + xsc0)) : 0.f;   // tokens past m: 0
-      const float sx1 = sx1_ok ? lds_f32(xsc_base + 4u * (blk * m_u + xsc1)) : 0.f;
       uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = make_uint4(0u, 0u, 0u, 0u);
       if (tok_ok) {
         xa = lds_v4(x_base + blk * 128u);
@@ -427,12 +428,29 @@ __global__ void __launch_bounds__(kLutThreads, 1) qlora_decode_lut_kernel(const 
       const uint32_t sbase = smem_u32(ring) + static_cast<uint32_t>(slot * slot_bytes);
       const uint32_t c1_row = static_cast<uint32_t>(c * kLutTile + g);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};   // rows g, g + 8 x tokens 2t, 2t + 1
+      const uint32_t cg_row = c1_base + 4u * c1_row * static_cast<uint32_t>(ss);
+      const uint32_t ch_row = cg_row + 4u * 8u * static_cast<uint32_t>(ss);
+      // one block with its scales loaded one by one (tokens past m: scale 0)
+      auto block1 = [&](int b) {
+        const uint32_t ub = static_cast<uint32_t>(b);
+        block(sbase, ub, lds_f32(cg_row + 4u * ub), lds_f32(ch_row + 4u * ub),
+              sx0_ok ? lds_f32(xsc_base + 4u * (xsc0 + ub)) : 0.f, sx1_ok ? lds_f32(xsc_base + 4u * (xsc1 + ub)) : 0.f,
+              acc);
+      };
       int blk = seg_lo;
-      for (; blk + 4 <= seg_hi; blk += 4) {   // four blocks at a time: offsets are immediates
-#pragma unroll
-        for (int q = 0; q < 4; ++q) block(sbase, static_cast<uint32_t>(blk + q), c1_row, acc);
+      for (; blk < seg_hi && (blk & 3) != 0; ++blk) block1(blk);
+      for (; blk + 4 <= seg_hi; blk += 4) {   // four blocks at a time: one 16-byte load per scale row
+        const uint32_t ub = static_cast<uint32_t>(blk);
+        const uint4 cg4 = lds_v4(cg_row + 4u * ub), ch4 = lds_v4(ch_row + 4u * ub);
+        uint4 s04 = make_uint4(0u, 0u, 0u, 0u), s14 = make_uint4(0u, 0u, 0u, 0u);
+        if (sx0_ok) s04 = lds_v4(xsc_base + 4u * (xsc0 + ub));
+        if (sx1_ok) s14 = lds_v4(xsc_base + 4u * (xsc1 + ub));
+        block(sbase, ub, __uint_as_float(cg4.x), __uint_as_float(ch4.x), __uint_as_float(s04.x), __uint_as_float(s14.x), acc);
+        block(sbase, ub + 1u, __uint_as_float(cg4.y), __uint_as_float(ch4.y), __uint_as_float(s04.y), __uint_as_float(s14.y), acc);
+        block(sbase, ub + 2u, __uint_as_float(cg4.z), __uint_as_float(ch4.z), __uint_as_float(s04.z), __uint_as_float(s14.z), acc);
+        block(sbase, ub + 3u, __uint_as_float(cg4.w), __uint_as_float(ch4.w), __uint_as_float(s04.w), __uint_as_float(s14.w), acc);
       }
-      for (; blk < seg_hi; ++blk) block(sbase, static_cast<uint32_t>(blk), c1_row, acc);
+      for (; blk < seg_hi; ++blk) block1(blk);
       // partial totals of this warp, [tile row][token][warp]; then the slot is free
       float* pt = part + static_cast<int64_t>(c * kLutTile) * m * kLutPartStride;
       if (2 * t < m) {
