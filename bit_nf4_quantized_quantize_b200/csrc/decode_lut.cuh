@@ -32,14 +32,18 @@
 //   multiplied by the inverse power of two together with c1.
 //
 // Work split: a CTA owns T tiles of 16 consecutive rows and all of K.  A
-// producer warp streams the tiles through a ring of shared-memory slots, one
-// bulk asynchronous copy per row into rows padded so that the consumers'
-// 8-byte operand loads never conflict, plus one copy of the 8-bit block
-// constants of all the CTA's rows.  The 16 compute warps work on one tile at
-// a time, each on its own range of 64-column blocks, and leave their partial
-// row totals in shared memory; the epilogue adds the 16 partials in warp
-// order (so the result does not depend on timing), adds s (U B^T) and writes
-// bf16 Y.
+// producer warp first copies the M token rows of X (bf16, one bulk copy per
+// token, into padded rows that the compute warps convert to scaled fp16 in
+// place) and the 8-bit block constants of all the CTA's rows, then streams
+// the tiles through a ring of shared-memory slots, one bulk asynchronous copy
+// per row into rows padded so that the consumers' 8-byte operand loads never
+// conflict.  The compute warps build the lookup table while those copies
+// land.  The c1 and activation-scale tables are stored by row with a stride
+// of 4 mod 32 floats, so one 16-byte load brings four blocks' scales of a row
+// without bank conflicts.  The 16 compute warps work on one tile at a time,
+// each on its own range of 64-column blocks, and leave their partial row
+// totals in shared memory; the epilogue adds the 16 partials in warp order
+// (so the result does not depend on timing), adds s (U B^T) and writes bf16 Y.
 //
 // Ordering.  qlora_decode_u_kernel (U = X A^T, launched just before this
 // kernel on the same stream) starts early, prefetches this kernel's weight
