@@ -204,9 +204,10 @@ size_t qlora_workspace_bytes(int64_t M, int64_t n_out, int64_t k_in, int r);
  * NF4 levels through a shared-memory table and applies c1 to each 64-column
  * block's fp32 dot product, so it multiplies by the fp32 dequantized value
  * level * c1 (to the level's fp16 rounding) rather than its bf16 rounding: a
- * difference of about 2^-9 of each weight, well within the layer's tolerance);
- * M <= 32, one (few-token
- * tensor-memory kernel); larger M, U and then the fused GEMM.
+ * difference of about 2^-9 of each weight, well within the layer's tolerance;
+ * shapes whose table-kernel shared memory would exceed 224 KiB take the next
+ * path instead); M <= 32, one (few-token tensor-memory kernel); larger M, U and
+ * then the fused GEMM.
  */
 int qlora_linear_fwd(const uint8_t* codes, const uint8_t* q8, const float* s2,
                      int64_t n_out, int64_t k_in,
