@@ -114,16 +114,17 @@ const Nf4Tables& tables() {
 constexpr int kMaxDevices = 64;
 
 int check_device(int* dev_out, int* num_sms) {
-  static int cached_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 bad
-  static int cached_sms[kMaxDevices];
+  // caches shared by host threads: cached_sms is written before cached_ok publishes it
+  static std::atomic<int> cached_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 bad
+  static std::atomic<int> cached_sms[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_NO_DEVICE; }
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_NO_DEVICE;
   if (cached_ok[dev] == 0) {
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_NO_DEVICE; }
-    cached_ok[dev] = (prop.major == 10) ? 1 : -1;
     cached_sms[dev] = prop.multiProcessorCount;
+    cached_ok[dev] = (prop.major == 10) ? 1 : -1;
   }
   if (cached_ok[dev] != 1) return QLORA_ERR_NO_DEVICE;
   *dev_out = dev;
@@ -246,7 +247,7 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
   auto kern = qlora_gemm_kernel<BN, NSTAGE, A_MN, BSRC, OUT, NDW, MH>;
   // the adapter slices must fit in the first pass over the stages
   if (args.n_lora > NSTAGE) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  static bool attr_set[kMaxDevices];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
       cudaGetLastError();
@@ -275,7 +276,7 @@ int launch_pair(int num_pairs, const CUtensorMap& a, const CUtensorMap& p, const
     return QLORA_ERR_CUDA;
   using L = PairSmem<MH>;
   auto kern = qlora_fused_pair_kernel<BSRC, MH>;
-  static bool attr_set[kMaxDevices];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
       cudaGetLastError();
@@ -300,8 +301,8 @@ int launch_decode(const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMa
                   DecodeArgs& d, cudaStream_t st, int dev) {
   using L = DecodeSmem<MP>;
   auto kern = qlora_decode_kernel<MP>;
-  static bool attr_set[kMaxDevices];
-  static int max_clusters[kMaxDevices][9];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
+  static std::atomic<int> max_clusters[kMaxDevices][9];
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
       cudaGetLastError();
@@ -427,7 +428,7 @@ int run_decode_lut(const uint8_t* codes, const uint8_t* q8, const float* s2, int
   u.consts_size = q8 ? 1 : 4;
   u.n = static_cast<int>(N);
   u.rows_per_cta = T * kLutTile;
-  static bool attr_set[kMaxDevices];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(qlora_decode_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutMaxSmem) !=
         cudaSuccess) {
@@ -552,7 +553,7 @@ int launch_lora(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap&
                 const LoraArgs& args, int tiles_total, int S, cudaStream_t st, int dev, int kind, int cx = 1) {
   auto kern = qlora_lora_kernel<A_MN, B_MN, STAGES, KB>;
   using L = LoraSmem<STAGES, KB>;
-  static bool attr_set[kMaxDevices];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) != cudaSuccess) {
       cudaGetLastError();
@@ -698,7 +699,7 @@ int launch_dropout_mask(const uint16_t* X, int64_t M, int64_t K, const DropoutSp
     cudaGetLastError();
     return QLORA_ERR_CUDA;
   }
-  static int resident[kMaxDevices];   // blocks of 256 threads per SM, 0 = not yet asked
+  static std::atomic<int> resident[kMaxDevices];   // blocks of 256 threads per SM, 0 = not yet asked
   if (resident[dev] == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dropout_mask_kernel, 256, 0) != cudaSuccess || n < 1) {
@@ -824,7 +825,7 @@ template <int kMode>
 int launch_quantize(int64_t groups, int sms, int dev, cudaStream_t st, const float* W, int64_t n_blocks,
                     uint8_t* codes, uint8_t* q8, float* s2) {
   auto kern = quantize_nf4_kernel<kMode>;
-  static bool attr_set[kMaxDevices];
+  static std::atomic<bool> attr_set[kMaxDevices];   // one-time setup done (stored last)
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(QuantSmem)) != cudaSuccess) {
       cudaGetLastError();
