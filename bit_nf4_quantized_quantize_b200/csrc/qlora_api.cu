@@ -176,7 +176,7 @@ struct TimingRec {
   cudaEvent_t start, stop;
 };
 std::mutex g_timing_mu;
-bool g_timing_on = false;
+std::atomic<bool> g_timing_on{false};   // read by every launch, set by qlora_timing_enable
 std::vector<TimingRec> g_timing_recs;
 std::vector<cudaEvent_t> g_event_pool;
 
